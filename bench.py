@@ -1,0 +1,447 @@
+"""Benchmark: one step = one pass of the whole block-sparse prefill path
+(block means -> pooled scores -> threshold mask -> sparse attention with the
+block-mean correction) over the 128K-token causal layer (Hq 32, Hkv 8, d 128,
+block 128, 80 % of causal block pairs dropped), seeded synthetic inputs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--dtype bf16|fp8|both]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, sampled
+
+Prints one JSON line (rank 0).  N > 1 runs one independent layer per GPU
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "128K prefill attn ms/layer & effective TFLOPS; % of B200 tensor peak"
+WORKLOAD_ID = 3
+DROP = 0.8
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="fp2", choices=["fp2", "reference"])
+    ap.add_argument("--dtype", default="both", choices=["bf16", "fp8", "both"])
+    ap.add_argument("--drop", type=float, default=DROP)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+# --------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed loop runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- work math ---
+def algorithmic_flops(cnt, lens_q, lens_k, B, d):
+    """Useful flops of the attention launch: exact-causal kept block pairs
+    (4*n_i*B*d per off-diagonal kept pair, 2*d*n_i*(n_i+1) for the diagonal
+    one) and the correction (4*d*n_i per dropped pair).  cnt: kept counts
+    [S, Hq, nqb_max] (forced blocks included)."""
+    kept_fl = 0.0
+    corr_fl = 0.0
+    dropped = 0
+    causal = 0
+    for b, (Lq, Lk) in enumerate(zip(lens_q, lens_k)):
+        nqb = -(-Lq // B)
+        pb = (Lk - Lq) // B
+        for i in range(nqb):
+            n_i = min(B, Lq - i * B)
+            iabs = pb + i
+            c = cnt[b, :, i].astype(np.float64)        # per head
+            off = c - 1.0                               # kept off-diagonal blocks
+            kept_fl += float(off.sum()) * 4.0 * n_i * B * d + c.size * 2.0 * d * n_i * (n_i + 1)
+            drop = (iabs + 1) - c
+            corr_fl += float(drop.sum()) * 4.0 * d * n_i
+            dropped += int(drop.sum())
+            causal += c.size * (iabs + 1)
+    return kept_fl, corr_fl, dropped / max(causal, 1)
+
+
+def dense_flops(lens_q, lens_k, Hq, d):
+    """Exact-causal dense flops: 4*d per (query, visible key) pair."""
+    f = 0.0
+    for Lq, Lk in zip(lens_q, lens_k):
+        P = Lk - Lq
+        f += 4.0 * d * Hq * (Lq * P + Lq * (Lq + 1) / 2.0)
+    return f
+
+
+# ---------------------------------------------------------------- GPU arm ---
+def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
+    import torch
+
+    from block_sparse_long_blockmean_b200 import fp2, synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shape = synth.workload(WORKLOAD_ID, dtype_name)
+    t0 = time.time()
+    inp = synth.make_inputs(shape)
+    gen_s = time.time() - t0
+    s = shape
+    dt = fp2.FP2_FP8_E4M3 if dtype_name == "fp8" else fp2.FP2_BF16
+    q = inp.q.to(dev)
+    k = inp.k.to(dev)
+    v = inp.v.to(dev)
+    cu = inp.cu_seqlens_q.to(dev)
+    lk = inp.seqlens_k.to(dev)
+    cuk = inp.cu_seqlens_k.to(dev)
+    sc = [x.to(dev) if x is not None else None for x in (inp.q_scale, inp.k_scale, inp.v_scale)]
+    stream = torch.cuda.Stream(dev)
+    pr = fp2.make_problem(q, k, v, cu, Hq=s.Hq, Hkv=s.Hkv, d=s.d, block=s.B, dtype=dt,
+                          max_seqlen_q=max(s.lens_q), max_seqlen_k=max(s.lens_k),
+                          seqlens_k=lk, cu_seqlens_k=cuk, q_scale=sc[0], k_scale=sc[1],
+                          v_scale=sc[2], stream=stream.cuda_stream)
+    P = pr.params
+    B = s.B
+    with torch.cuda.stream(stream):
+        # tau for the target drop, from this GPU's own scores (not timed)
+        fp2.blockmean(k, v, None, cu, B, dt, P)
+        fp2.score(q, cu, B, dt, P)
+        tau = fp2.calibrate_tau(cu, B, args.drop, P)
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            fp2.blockmean(k, v, None, cu, B, dt, P)
+            if ev is not None:
+                ev[1].record(stream)
+            fp2.score(q, cu, B, dt, P)
+            if ev is not None:
+                ev[2].record(stream)
+            fp2.mask(cu, tau, B, P)
+            if ev is not None:
+                ev[3].record(stream)
+            fp2.attn(q, k, v, None, cu, None, B, dt, pr.out, P)
+            if ev is not None:
+                ev[4].record(stream)
+
+        for _ in range(args.warmup):
+            step()
+        stream.synchronize()
+        pr.check()
+        L = pr.layout()
+        cnt = pr.ws_view("kept_cnt", torch.int32, (inp.num_seqs, s.Hq, L.nqb_max)).cpu().numpy()
+        kept_fl, corr_fl, drop_frac = algorithmic_flops(cnt, s.lens_q, s.lens_k, B, s.d)
+
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        clocks = ClockSampler(dev.index if dev.index is not None else 0)
+        clocks.start()
+        time.sleep(0.3)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for it in range(args.steps):
+            step(evs[it])
+        end.record(stream)
+        stream.synchronize()
+        clk = clocks.stop()
+        torch.cuda.synchronize()
+        pr.check()
+        total_ms = start.elapsed_time(end)
+        stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
+                          for i in range(args.steps)])
+        stage_ms = stage.mean(axis=0)
+
+        dense = None
+        if not args.no_dense:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            fp2.mask(cu, math.inf, B, P)
+            fp2.attn(q, k, v, None, cu, None, B, dt, pr.out, P)  # warm
+            e0.record(stream)
+            fp2.attn(q, k, v, None, cu, None, B, dt, pr.out, P)
+            e1.record(stream)
+            stream.synchronize()
+            dense = {"attn_ms": e0.elapsed_time(e1),
+                     "tflops": dense_flops(s.lens_q, s.lens_k, s.Hq, s.d) / (e0.elapsed_time(e1) * 1e-3) / 1e12}
+            fp2.mask(cu, tau, B, P)
+
+        e2e = None
+        if not args.no_e2e:
+            # through the public API with HOST buffers: H2D of q, k, v from
+            # pinned memory, fp2_prefill, D2H of the output, every step
+            hq = inp.q.pin_memory()
+            hk = inp._kc.pin_memory()
+            hv = inp._vc.pin_memory()
+            hout = torch.empty(pr.out.shape, dtype=torch.bfloat16).pin_memory()
+            nsteps = max(2, min(args.steps, 5))
+            for it in range(nsteps + 1):
+                if it == 1:
+                    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    ea.record(stream)
+                q.copy_(hq, non_blocking=True)
+                k.copy_(hk, non_blocking=True)
+                v.copy_(hv, non_blocking=True)
+                fp2.prefill(q, k, v, None, cu, tau, B, dt, pr.out, P)
+                hout.copy_(pr.out, non_blocking=True)
+            eb.record(stream)
+            stream.synchronize()
+            pr.check()
+            e2e_ms = ea.elapsed_time(eb) / nsteps
+            e2e = {"value": e2e_ms, "unit": "ms/layer",
+                   "h2d_bytes_per_step": int(hq.numel() * hq.element_size() +
+                                             hk.numel() * hk.element_size() +
+                                             hv.numel() * hv.element_size()),
+                   "d2h_bytes_per_step": int(hout.numel() * hout.element_size())}
+    res = {
+        "dtype": dtype_name, "tau": tau, "drop_fraction": drop_frac,
+        "total_ms": total_ms, "ms_per_step": total_ms / args.steps,
+        "stage_ms": {"blockmean": stage_ms[0], "score": stage_ms[1], "mask": stage_ms[2],
+                     "attn": stage_ms[3]},
+        "kept_flops": kept_fl, "corr_flops": corr_fl, "clocks": clk, "dense": dense,
+        "e2e": e2e, "gen_s": gen_s, "inp": inp if want_cpu else None, "tau_inp": tau,
+    }
+    return res
+
+
+def cpu_baseline(inp, tau, budget_blocks=4, heads_per_block=8):
+    """The fp64 oracle on a bounded sample of the same layer: every block
+    mean, pooled score and mask of the whole layer, then the corrected
+    attention of `heads_per_block` heads x all rows of `budget_blocks` query
+    blocks at evenly spaced depths; the attention time is scaled to all
+    blocks and heads (its cost grows linearly with the block index)."""
+    from oracle import oracle as O
+    s = inp.shape
+    B = s.B
+    t0 = time.time()
+    K, V = inp.seq_k(0), inp.seq_v(0)
+    kbar, vbar, cnt = O.blockmean(K, V, B)
+    Lq = s.lens_q[0]
+    nqb = -(-Lq // B)
+    parts = []
+    for i0 in range(0, nqb, 64):
+        Qc = inp._deq(inp.q[i0 * B: min(Lq, (i0 + 64) * B)], inp.q_scale)
+        parts.append(O.pool_q(Qc, B))
+    qbar = np.concatenate(parts, axis=1)
+    S = O.score(qbar, kbar, 0)
+    keep = O.mask(S, 0, tau)
+    t_sel = time.time() - t0
+    blocks = [int((m + 0.5) * nqb / budget_blocks) for m in range(budget_blocks)]
+    heads = np.arange(heads_per_block, dtype=np.int32)
+    t1 = time.time()
+    for i in blocks:
+        Qb = inp._deq(inp.q[i * B: min(Lq, (i + 1) * B)], inp.q_scale)
+        O.attn_query_block(Qb, K, V, kbar, vbar, cnt, keep[:, i], B, i, heads)
+    t_attn = time.time() - t1
+    scale = (nqb / budget_blocks) * (s.Hq / heads_per_block)
+    est_s = t_sel + t_attn * scale
+    return {"value": est_s * 1e3, "unit": "ms/layer", "cores": O.num_threads(), "kind": "oracle",
+            "sample": (f"whole-layer block means, pooled scores and mask ({t_sel:.1f} s) + "
+                       f"corrected attention of {heads_per_block}/{s.Hq} heads x "
+                       f"{budget_blocks}/{nqb} query blocks ({t_attn:.1f} s), "
+                       f"attention scaled x{scale:.0f}")}
+
+
+def reference_arm(args):
+    """--impl reference: the fp64 CPU oracle as it stands, each step a bounded
+    sample of the same layer (one query block x 4 heads), scaled to ms/layer."""
+    from block_sparse_long_blockmean_b200 import synth
+    from oracle import oracle as O
+    shape = synth.workload(WORKLOAD_ID, "bf16")
+    inp = synth.make_inputs(shape)
+    s = shape
+    B = s.B
+    K, V = inp.seq_k(0), inp.seq_v(0)
+    kbar, vbar, cnt = O.blockmean(K, V, B)
+    Lq = s.lens_q[0]
+    nqb = -(-Lq // B)
+    parts = []
+    for i0 in range(0, nqb, 64):
+        parts.append(O.pool_q(inp._deq(inp.q[i0 * B: (i0 + 64) * B], None), B))
+    S = O.score(np.concatenate(parts, axis=1), kbar, 0)
+    tau = O.tau_for_drop([S], [0], args.drop)
+    keep = O.mask(S, 0, tau)
+    rng = np.random.default_rng(0)
+    times = []
+    heads = np.arange(4, dtype=np.int32)
+    kept_all = keep.sum()
+    for it in range(args.warmup + args.steps):
+        i = int(rng.integers(0, nqb))
+        Qb = inp._deq(inp.q[i * B: (i + 1) * B], None)
+        t0 = time.time()
+        O.attn_query_block(Qb, K, V, kbar, vbar, cnt, keep[:, i], B, i, heads)
+        dt = time.time() - t0
+        # the cost of a block grows with its kept blocks; scale to the layer
+        kept_i = keep[:4, i].sum()
+        if it >= args.warmup:
+            times.append(dt * kept_all / max(kept_i, 1))
+    ms = float(np.mean(times)) * 1e3
+    line = {"metric": METRIC, "value": ms, "unit": "ms/layer", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": synth.WORKLOAD_NAMES[WORKLOAD_ID], "drop": args.drop},
+            "cpu_baseline": {"value": ms, "unit": "ms/layer", "cores": O.num_threads(),
+                             "kind": "oracle",
+                             "sample": "per step: corrected attention of 4 heads x 1 random "
+                                       "query block, scaled by kept-block count to the layer"},
+            "e2e": {"value": ms, "unit": "ms/layer", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        if rank == 0:
+            reference_arm(args)
+        return
+    import torch
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    from block_sparse_long_blockmean_b200 import fp2, synth
+    fp2.lib()
+    peaks, peak_src = measured_peaks()
+    dtypes = ["bf16", "fp8"] if args.dtype == "both" else [args.dtype]
+    results = {}
+    for dn in dtypes:
+        results[dn] = run_gpu(args, rank, world, dn, want_cpu=(dn == dtypes[0]))
+    main_dt = dtypes[0]
+    r = results[main_dt]
+    total_ms = r["total_ms"]
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_layer = total_ms / (args.steps * world)
+
+    def summary(x):
+        attn_ms = x["stage_ms"]["attn"]
+        eff = x["kept_flops"] / (attn_ms * 1e-3) / 1e12
+        bf16_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        peak = bf16_peak * (2.0 if x["dtype"] == "fp8" else 1.0)
+        out = {"attn_ms": attn_ms, "ms_per_layer": x["ms_per_step"],
+               "eff_tflops_kept": eff,
+               "eff_tflops_incl_correction": (x["kept_flops"] + x["corr_flops"]) / (attn_ms * 1e-3) / 1e12,
+               "tensor_peak_frac_measured": eff / peak,
+               "tensor_peak_frac_datasheet": eff / (2250.0 * (2.0 if x["dtype"] == "fp8" else 1.0)),
+               "drop_fraction": x["drop_fraction"], "tau": x["tau"],
+               "stage_ms": x["stage_ms"],
+               "prefill_roofline_frac": (x["kept_flops"] / peak / 1e12) / (x["ms_per_step"] * 1e-3)}
+        if x["dense"]:
+            out["dense_attn_ms"] = x["dense"]["attn_ms"]
+            out["dense_tflops"] = x["dense"]["tflops"]
+            out["speedup_vs_own_dense_attn"] = x["dense"]["attn_ms"] / attn_ms
+        return out, peak
+
+    s_main, peak = summary(r)
+    eff = s_main["eff_tflops_kept"]
+    line = {
+        "metric": METRIC, "value": ms_per_layer, "unit": "ms/layer", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": main_dt,
+        "data": "synthetic",
+        "config": {"workload": synth.WORKLOAD_NAMES[WORKLOAD_ID], "seq_len": 131072,
+                   "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128, "block": 128,
+                   "target_drop": args.drop, "layout": "contiguous K/V",
+                   "l2": "inputs (1.6 GB) larger than L2; no flush",
+                   "per_gpu": "one independent layer per GPU"},
+        "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
+                     "frac": eff / peak, "traffic": None,
+                     "kernel": "fp2_attn (attn_kernel)",
+                     "peak_source": f"{peak_src} bf16_tflops_sustained" +
+                                    (" x2 (fp8/bf16 nominal ratio)" if main_dt == "fp8" else "")},
+        "summary": {main_dt: s_main},
+        "gpu_launches": 4 * args.steps,
+        "clocks": r["clocks"],
+    }
+    for dn in dtypes[1:]:
+        line["summary"][dn] = summary(results[dn])[0]
+    if r["e2e"]:
+        line["e2e"] = r["e2e"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(r["inp"], r["tau"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,330 @@
+// fp2_api.cu -- the C ABI of include/fp2.h: argument validation, workspace
+// layout, stream-ordered launches of the four kernels, status read-back and
+// the host-side tau calibration utility.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "fp2.h"
+#include "fp2_internal.h"
+
+using fp2::KParams;
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+fp2_status check_params(const fp2_params* P, int block) {
+    if (!P) return FP2_ERR_INVALID_ARG;
+    if (P->num_seqs < 1 || P->num_q_heads < 1 || P->num_kv_heads < 1 || P->total_q < 0 ||
+        P->max_seqlen_q < 0 || P->max_seqlen_k < P->max_seqlen_q || P->max_seqlen_k < 1)
+        return FP2_ERR_INVALID_ARG;
+    if (P->num_q_heads % P->num_kv_heads != 0) return FP2_ERR_INVALID_ARG;
+    const int G = P->num_q_heads / P->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return FP2_ERR_UNSUPPORTED;
+    if (P->head_dim != 64 && P->head_dim != 128) return FP2_ERR_UNSUPPORTED;
+    if (block != 64 && block != 128) return FP2_ERR_UNSUPPORTED;
+    if (128 / G > block) return FP2_ERR_UNSUPPORTED;
+    return FP2_OK;
+}
+
+fp2_status check_kv(const fp2_params* P, int block, const int32_t* page_table) {
+    if (page_table) {
+        if (!is_pow2(P->page_size) || P->page_size < 16 || P->page_size > 256)
+            return FP2_ERR_UNSUPPORTED;
+        if (block % P->page_size != 0 && P->page_size % block != 0) return FP2_ERR_UNSUPPORTED;
+        if (P->max_pages_per_seq < 1 || P->num_pages < 1) return FP2_ERR_INVALID_ARG;
+    } else {
+        if (P->total_k < 0) return FP2_ERR_INVALID_ARG;
+    }
+    return FP2_OK;
+}
+
+fp2_status check_dtype(const fp2_params* P, int block, fp2_dtype dtype) {
+    if (dtype == FP2_BF16) return FP2_OK;
+    if (dtype != FP2_FP8_E4M3) return FP2_ERR_INVALID_ARG;
+    if (P->head_dim != 128 || block != 128) return FP2_ERR_UNSUPPORTED;
+    if (!P->q_scale || !P->k_scale || !P->v_scale) return FP2_ERR_INVALID_ARG;
+    return FP2_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void layout_of(const fp2_params* P, int block, fp2_workspace_layout* L) {
+    const size_t S = (size_t)P->num_seqs, Hq = (size_t)P->num_q_heads,
+                 Hkv = (size_t)P->num_kv_heads, d = (size_t)P->head_dim;
+    const int nqb = (P->max_seqlen_q + block - 1) / block;
+    const int nkb = (P->max_seqlen_k + block - 1) / block;
+    const int nw = (nkb + 31) / 32;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + bytes, 256);
+        return at;
+    };
+    L->error_word = take(256);
+    L->kbar = take(S * Hkv * nkb * d * 4);
+    L->vbar = take(S * Hkv * nkb * d * 4);
+    L->kbar_op = take(S * Hkv * nkb * d * 2);
+    L->vbar_op = take(S * Hkv * nkb * d * 2);
+    L->scores = take(S * Hq * nqb * nkb * 4);
+    L->kept_idx = take(S * Hq * nqb * nkb * 4);
+    L->kept_cnt = take(S * Hq * nqb * 4);
+    L->kept_bits = take(S * Hq * nqb * nw * 4);
+    L->total = o;
+    L->nqb_max = nqb;
+    L->nkb_max = nkb;
+    L->nw = nw;
+}
+
+// Validates what every entry point needs and fills the kernel parameters.
+fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_t* cu_seqlens,
+                   const int32_t* page_table, KParams& kp, bool uses_kv = true) {
+    fp2_status st = check_params(P, block);
+    if (st != FP2_OK) return st;
+    if ((st = check_dtype(P, block, dtype)) != FP2_OK) return st;
+    if ((st = check_kv(P, block, page_table)) != FP2_OK) return st;
+    if (!cu_seqlens) return FP2_ERR_INVALID_ARG;
+    fp2_workspace_layout L;
+    layout_of(P, block, &L);
+    if (!P->workspace || (reinterpret_cast<uintptr_t>(P->workspace) & 255u) != 0 ||
+        P->workspace_bytes < L.total)
+        return FP2_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(P->workspace);
+    std::memset(&kp, 0, sizeof(kp));
+    kp.num_seqs = P->num_seqs;
+    kp.Hq = P->num_q_heads;
+    kp.Hkv = P->num_kv_heads;
+    kp.d = P->head_dim;
+    kp.G = kp.Hq / kp.Hkv;
+    kp.B = block;
+    kp.total_q = P->total_q;
+    kp.total_k = P->total_k;
+    kp.paged = page_table ? 1 : 0;
+    kp.page_size = page_table ? P->page_size : 0;
+    kp.max_pages = page_table ? P->max_pages_per_seq : 0;
+    kp.num_pages = page_table ? P->num_pages : 0;
+    kp.max_seqlen_q = P->max_seqlen_q;
+    kp.max_seqlen_k = P->max_seqlen_k;
+    kp.nqb_max = L.nqb_max;
+    kp.nkb_max = L.nkb_max;
+    kp.nw = L.nw;
+    kp.fp8 = dtype == FP2_FP8_E4M3;
+    kp.uses_kv = uses_kv ? 1 : 0;
+    kp.cu_q = cu_seqlens;
+    kp.cu_k = P->cu_seqlens_k ? P->cu_seqlens_k : cu_seqlens;
+    kp.seqlens_k = P->seqlens_k;
+    kp.page_table = page_table;
+    kp.q_scale = P->q_scale;
+    kp.k_scale = P->k_scale;
+    kp.v_scale = P->v_scale;
+    kp.err = reinterpret_cast<uint32_t*>(ws + L.error_word);
+    kp.kbar = reinterpret_cast<float*>(ws + L.kbar);
+    kp.vbar = reinterpret_cast<float*>(ws + L.vbar);
+    kp.kbar_op = ws + L.kbar_op;
+    kp.vbar_op = ws + L.vbar_op;
+    kp.scores = reinterpret_cast<float*>(ws + L.scores);
+    kp.kept_idx = reinterpret_cast<int32_t*>(ws + L.kept_idx);
+    kp.kept_cnt = reinterpret_cast<int32_t*>(ws + L.kept_cnt);
+    kp.kept_bits = reinterpret_cast<uint32_t*>(ws + L.kept_bits);
+    return FP2_OK;
+}
+
+cudaStream_t stream_of(const fp2_params* P) { return static_cast<cudaStream_t>(P->stream); }
+
+fp2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP2_OK : FP2_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* fp2_version(void) { return "0.1.0"; }
+
+const char* fp2_status_string(fp2_status s) {
+    switch (s) {
+        case FP2_OK: return "ok";
+        case FP2_ERR_INVALID_ARG: return "invalid argument";
+        case FP2_ERR_UNSUPPORTED: return "unsupported configuration";
+        case FP2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case FP2_ERR_CUDA: return "CUDA error";
+        case FP2_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case FP2_ERR_DEVICE_BOUNDS: return "device index out of range";
+    }
+    return "unknown status";
+}
+
+size_t fp2_workspace_size(const fp2_params* params, int block) {
+    if (check_params(params, block) != FP2_OK) return 0;
+    fp2_workspace_layout L;
+    layout_of(params, block, &L);
+    return L.total;
+}
+
+fp2_status fp2_get_workspace_layout(const fp2_params* params, int block,
+                                    fp2_workspace_layout* layout) {
+    if (!layout) return FP2_ERR_INVALID_ARG;
+    fp2_status st = check_params(params, block);
+    if (st != FP2_OK) return st;
+    layout_of(params, block, layout);
+    return FP2_OK;
+}
+
+fp2_status fp2_blockmean(const void* k_cache, const void* v_cache, const int32_t* page_table,
+                         const int32_t* cu_seqlens, int block, fp2_dtype dtype,
+                         const fp2_params* params) {
+    KParams kp;
+    fp2_status st = prepare(params, block, dtype, cu_seqlens, page_table, kp);
+    if (st != FP2_OK) return st;
+    if (!k_cache || !v_cache) return FP2_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return FP2_ERR_INVALID_ARG;
+    return cuda_status(fp2::launch_blockmean(kp, k_cache, v_cache, stream_of(params)));
+}
+
+fp2_status fp2_score(const void* q, const int32_t* cu_seqlens, int block, fp2_dtype dtype,
+                     const fp2_params* params) {
+    KParams kp;
+    fp2_status st = prepare(params, block, dtype, cu_seqlens, nullptr, kp, false);
+    if (st != FP2_OK) return st;
+    if (!q || !aligned16(q)) return FP2_ERR_INVALID_ARG;
+    return cuda_status(fp2::launch_score(kp, q, stream_of(params)));
+}
+
+fp2_status fp2_mask(const int32_t* cu_seqlens, float tau, int block, const fp2_params* params) {
+    KParams kp;
+    fp2_status st = prepare(params, block, FP2_BF16, cu_seqlens, nullptr, kp, false);
+    if (st != FP2_OK) return st;
+    if (std::isnan(tau)) return FP2_ERR_INVALID_ARG;
+    return cuda_status(fp2::launch_mask(kp, tau, stream_of(params)));
+}
+
+fp2_status fp2_attn(const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* page_table, const int32_t* cu_seqlens,
+                    const uint32_t* kept_bits, int block, fp2_dtype dtype, void* out,
+                    const fp2_params* params) {
+    KParams kp;
+    fp2_status st = prepare(params, block, dtype, cu_seqlens, page_table, kp);
+    if (st != FP2_OK) return st;
+    if (!q || !k_cache || !v_cache || !out) return FP2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return FP2_ERR_INVALID_ARG;
+    if (kp.total_q == 0) return FP2_OK;
+    if (!page_table && kp.total_k == 0) return FP2_ERR_INVALID_ARG;
+    const uint32_t* bits = kept_bits ? kept_bits : kp.kept_bits;
+    cudaError_t e = fp2::launch_attn(kp, q, k_cache, v_cache, bits, out, stream_of(params));
+    if (e == cudaErrorInvalidValue) return FP2_ERR_UNSUPPORTED;
+    return cuda_status(e);
+}
+
+fp2_status fp2_prefill(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* page_table, const int32_t* cu_seqlens, float tau,
+                       int block, fp2_dtype dtype, void* out, const fp2_params* params) {
+    KParams kp;
+    fp2_status st = prepare(params, block, dtype, cu_seqlens, page_table, kp);
+    if (st != FP2_OK) return st;
+    if (!q || !k_cache || !v_cache || !out) return FP2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return FP2_ERR_INVALID_ARG;
+    if (std::isnan(tau)) return FP2_ERR_INVALID_ARG;
+    if (kp.total_q == 0) return FP2_OK;
+    if (!page_table && kp.total_k == 0) return FP2_ERR_INVALID_ARG;
+    cudaStream_t s = stream_of(params);
+    cudaError_t e = fp2::launch_blockmean(kp, k_cache, v_cache, s);
+    if (e == cudaSuccess) e = fp2::launch_score(kp, q, s);
+    if (e == cudaSuccess) e = fp2::launch_mask(kp, tau, s);
+    if (e == cudaSuccess) e = fp2::launch_attn(kp, q, k_cache, v_cache, kp.kept_bits, out, s);
+    if (e == cudaErrorInvalidValue) return FP2_ERR_UNSUPPORTED;
+    return cuda_status(e);
+}
+
+fp2_status fp2_workspace_init(const fp2_params* params) {
+    if (!params || !params->workspace || params->workspace_bytes < 256) return FP2_ERR_WORKSPACE;
+    return cuda_status(cudaMemsetAsync(params->workspace, 0, 256, stream_of(params)));
+}
+
+fp2_status fp2_get_status(const fp2_params* params, uint32_t* detail) {
+    if (!params || !params->workspace) return FP2_ERR_INVALID_ARG;
+    cudaStream_t s = stream_of(params);
+    uint32_t w[2] = {0, 0};
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FP2_ERR_CUDA;
+    if (cudaMemcpy(w, params->workspace, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FP2_ERR_CUDA;
+    if (w[0] != 0) {
+        if (cudaMemsetAsync(params->workspace, 0, sizeof(w), s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return FP2_ERR_CUDA;
+    }
+    if (detail) *detail = w[1];
+    return static_cast<fp2_status>(w[0]);
+}
+
+fp2_status fp2_calibrate_tau(const int32_t* cu_seqlens, int block, float target_drop,
+                             const fp2_params* params, float* tau_out) {
+    KParams kp;
+    fp2_status st = prepare(params, block, FP2_BF16, cu_seqlens, nullptr, kp, false);
+    if (st != FP2_OK) return st;
+    if (!tau_out || !(target_drop >= 0.f && target_drop <= 1.f)) return FP2_ERR_INVALID_ARG;
+    cudaStream_t s = stream_of(params);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FP2_ERR_CUDA;
+    const int S = kp.num_seqs;
+    std::vector<int32_t> cu(S + 1), lk(S);
+    if (cudaMemcpy(cu.data(), cu_seqlens, (S + 1) * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FP2_ERR_CUDA;
+    if (kp.seqlens_k) {
+        if (cudaMemcpy(lk.data(), kp.seqlens_k, S * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return FP2_ERR_CUDA;
+    } else {
+        for (int b = 0; b < S; ++b) lk[b] = cu[b + 1] - cu[b];
+    }
+    std::vector<double> margins;
+    size_t total = 0;
+    std::vector<float> slab((size_t)kp.nqb_max * kp.nkb_max);
+    for (int b = 0; b < S; ++b) {
+        const int Lq = cu[b + 1] - cu[b];
+        if (Lq < 0 || Lq > kp.max_seqlen_q || lk[b] < Lq || lk[b] > kp.max_seqlen_k ||
+            (lk[b] - Lq) % block != 0)
+            return FP2_ERR_INVALID_ARG;
+        const int pb = (lk[b] - Lq) / block;
+        const int nqb = (Lq + block - 1) / block;
+        for (int h = 0; h < kp.Hq; ++h) {
+            const size_t off = ((size_t)b * kp.Hq + h) * kp.nqb_max * kp.nkb_max;
+            if (cudaMemcpy(slab.data(), kp.scores + off, (size_t)nqb * kp.nkb_max * 4,
+                           cudaMemcpyDeviceToHost) != cudaSuccess)
+                return FP2_ERR_CUDA;
+            for (int i = 0; i < nqb; ++i) {
+                const int iabs = pb + i;
+                const float* row = slab.data() + (size_t)i * kp.nkb_max;
+                total += (size_t)iabs + 1;
+                double m = -INFINITY;
+                for (int j = 0; j <= iabs; ++j) m = std::max(m, (double)row[j]);
+                for (int j = 1; j < iabs; ++j) margins.push_back(m - (double)row[j]);
+            }
+        }
+    }
+    const size_t n = margins.size();
+    if (n == 0) {
+        *tau_out = INFINITY;
+        return FP2_OK;
+    }
+    long long want = std::llround((double)target_drop * (double)total);
+    want = std::max(0LL, std::min<long long>(want, (long long)n));
+    if (want == 0) {
+        *tau_out = (float)(*std::max_element(margins.begin(), margins.end()) + 1.0);
+        return FP2_OK;
+    }
+    if (want == (long long)n) {
+        const double lo = *std::min_element(margins.begin(), margins.end());
+        *tau_out = (float)(lo > 0 ? lo / 2 : lo - 1.0);
+        return FP2_OK;
+    }
+    const size_t k = n - (size_t)want;  // tau between the k-th and (k+1)-th smallest
+    std::nth_element(margins.begin(), margins.begin() + k, margins.end());
+    const double hi = margins[k];
+    const double lo = *std::max_element(margins.begin(), margins.begin() + k);
+    *tau_out = (float)(0.5 * (lo + hi));
+    return FP2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,53 @@
+// fp2_internal.h -- parameter block shared by the host launcher and the
+// kernels of the fp2 library (not part of the public ABI).
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime.h>
+
+namespace fp2 {
+
+struct KParams {
+    int num_seqs, Hq, Hkv, d, G, B;
+    int total_q, total_k;
+    int paged, page_size, max_pages, num_pages;
+    int max_seqlen_q, max_seqlen_k;
+    int nqb_max, nkb_max, nw;
+    int fp8;
+    int uses_kv;               // 0: the launch never reads K/V (no key-extent check)
+    const int32_t* cu_q;       // [S+1]
+    const int32_t* cu_k;       // [S+1] contiguous key offsets (may alias cu_q)
+    const int32_t* seqlens_k;  // [S] or nullptr
+    const int32_t* page_table; // [S][max_pages] or nullptr
+    const float* q_scale;
+    const float* k_scale;
+    const float* v_scale;
+    uint32_t* err;             // error word (workspace)
+    float* kbar;               // [S][Hkv][nkb_max][d]
+    float* vbar;
+    void* kbar_op;             // bf16 | e4m3, same shape
+    void* vbar_op;
+    float* scores;             // [S][Hq][nqb_max][nkb_max]
+    int32_t* kept_idx;         // [S][Hq][nqb_max][nkb_max]
+    int32_t* kept_cnt;         // [S][Hq][nqb_max]
+    uint32_t* kept_bits;       // [S][Hq][nqb_max][nw]
+};
+
+// Detail codes stored beside an error code.
+enum : uint32_t {
+    kDetSeqLen = 1,      // Lq or Lk outside [0, max_seqlen_*] or Lk < Lq
+    kDetPrefix = 2,      // (Lk - Lq) % block != 0
+    kDetPage = 3,        // page id outside [0, num_pages)
+    kDetWaitBase = 16,   // + pipeline wait site
+};
+
+// Launchers (fp2_stages.cu, fp2_attn.cu).  Return the launch error.
+cudaError_t launch_blockmean(const KParams& p, const void* k, const void* v, cudaStream_t s);
+cudaError_t launch_score(const KParams& p, const void* q, cudaStream_t s);
+cudaError_t launch_mask(const KParams& p, float tau, cudaStream_t s);
+cudaError_t launch_attn(const KParams& p, const void* q, const void* k, const void* v,
+                        const uint32_t* kept_bits, void* out, cudaStream_t s);
+
+}  // namespace fp2

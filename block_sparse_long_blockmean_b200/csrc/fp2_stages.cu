@@ -1,0 +1,296 @@
+// fp2_stages.cu -- the three selection stages of FlashPrefill V2 on sm_100a:
+//   blockmean: per-block means of K and V ("V_avg_dropped" of the popular
+//              explainer, section 2.1) -- HBM-bound streaming reduction;
+//   score:     pooled query blocks dotted with every causal key-block mean
+//              (abstract: instantaneous pattern discovery) -- HBM-bound on Q;
+//   mask:      max-based dynamic threshold with block 0 and the diagonal
+//              always kept (abstract) -- one warp per (sequence, head, block).
+// All three move 16-byte vectors and reduce with warp shuffles or a small
+// shared-memory tree; none needs a tensor core.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "fp2_seq.cuh"
+
+namespace fp2 {
+
+template <bool FP8>
+__device__ __forceinline__ void unpack16(const uint4& v, float* out) {
+    if constexpr (FP8) {
+        const uint8_t* b = reinterpret_cast<const uint8_t*>(&v);
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+            __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(b[e] | (b[e + 1] << 8));
+            __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+            float2 f = __half22float2(*reinterpret_cast<__half2*>(&h));
+            out[e] = f.x;
+            out[e + 1] = f.y;
+        }
+    } else {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(h[e]);
+            out[2 * e] = f.x;
+            out[2 * e + 1] = f.y;
+        }
+    }
+}
+
+// ------------------------------------------------------------- blockmean ---
+// grid (nkb_max, Hkv, num_seqs), 128 threads.  Each CTA averages the valid
+// rows of one key block of one KV head, for K and V.  Blocks past the end
+// of the sequence are written as zeros (the attention kernel reads whole
+// tiles of means and multiplies the unused ones by zero).
+template <int D, bool FP8>
+__global__ void __launch_bounds__(128) blockmean_kernel(KParams p, const uint8_t* __restrict__ K,
+                                                        const uint8_t* __restrict__ V) {
+    constexpr int ELT = FP8 ? 1 : 2;
+    constexpr int VEC = 16 / ELT;   // elements per 16-byte load
+    constexpr int TPR = D / VEC;    // threads per row
+    constexpr int RPP = 128 / TPR;  // rows per pass
+    __shared__ float red[2][RPP][D];
+
+    const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    SeqInfo s;
+    if (!load_seq(p, b, s)) return;
+    const int nkb = (s.Lk + p.B - 1) / p.B;
+    const size_t orow = (((size_t)b * p.Hkv + hk) * p.nkb_max + j) * D;
+    if (j >= nkb) {
+        for (int c = threadIdx.x; c < D; c += 128) {
+            p.kbar[orow + c] = 0.f;
+            p.vbar[orow + c] = 0.f;
+            if constexpr (FP8) {
+                reinterpret_cast<uint8_t*>(p.kbar_op)[orow + c] = 0;
+                reinterpret_cast<uint8_t*>(p.vbar_op)[orow + c] = 0;
+            } else {
+                reinterpret_cast<__nv_bfloat16*>(p.kbar_op)[orow + c] = __float2bfloat16(0.f);
+                reinterpret_cast<__nv_bfloat16*>(p.vbar_op)[orow + c] = __float2bfloat16(0.f);
+            }
+        }
+        return;
+    }
+    const int t0 = j * p.B;
+    const int n = min(p.B, s.Lk - t0);
+    const int lv = threadIdx.x % TPR, rg = threadIdx.x / TPR;
+    float ak[VEC], av[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) ak[e] = av[e] = 0.f;
+    for (int r = rg; r < n; r += RPP) {
+        const long long row = key_row(p, s, b, t0 + r);
+        if (row < 0) continue;
+        const size_t off = ((size_t)row * p.Hkv + hk) * D * ELT + (size_t)lv * 16;
+        const uint4 kv = __ldg(reinterpret_cast<const uint4*>(K + off));
+        const uint4 vv = __ldg(reinterpret_cast<const uint4*>(V + off));
+        float fk[VEC], fv[VEC];
+        unpack16<FP8>(kv, fk);
+        unpack16<FP8>(vv, fv);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            ak[e] += fk[e];
+            av[e] += fv[e];
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        red[0][rg][lv * VEC + e] = ak[e];
+        red[1][rg][lv * VEC + e] = av[e];
+    }
+    __syncthreads();
+    const float inv = 1.f / (float)n;
+    const float ks = FP8 ? p.k_scale[hk] : 1.f;
+    const float vs = FP8 ? p.v_scale[hk] : 1.f;
+    for (int c = threadIdx.x; c < D; c += 128) {
+        float sk = 0.f, sv = 0.f;
+#pragma unroll
+        for (int r = 0; r < RPP; ++r) {
+            sk += red[0][r][c];
+            sv += red[1][r][c];
+        }
+        const float mk = sk * inv, mv = sv * inv;  // mean of the stored values
+        p.kbar[orow + c] = mk * ks;                // dequantised
+        p.vbar[orow + c] = mv * vs;
+        if constexpr (FP8) {
+            reinterpret_cast<__nv_fp8_e4m3*>(p.kbar_op)[orow + c] = __nv_fp8_e4m3(mk);
+            reinterpret_cast<__nv_fp8_e4m3*>(p.vbar_op)[orow + c] = __nv_fp8_e4m3(mv);
+        } else {
+            reinterpret_cast<__nv_bfloat16*>(p.kbar_op)[orow + c] = __float2bfloat16(mk);
+            reinterpret_cast<__nv_bfloat16*>(p.vbar_op)[orow + c] = __float2bfloat16(mv);
+        }
+    }
+}
+
+// ----------------------------------------------------------------- score ---
+// grid (nqb_max, Hkv, num_seqs), 256 threads.  Pools the valid rows of one
+// query block for the G query heads of one KV head (their rows are
+// contiguous in q), then one warp per key block j <= i_abs forms the G dot
+// products with kbar_j (lanes across d, shuffle reduction).
+template <int D, bool FP8, int G>
+__global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __restrict__ Q) {
+    constexpr int ELT = FP8 ? 1 : 2;
+    constexpr int VEC = 16 / ELT;
+    constexpr int VPT = G * D / VEC;          // 16-byte vectors per token (G heads)
+    constexpr int TPP = 256 / VPT;            // tokens per pass
+    static_assert(VPT <= 256 && 256 % VPT == 0, "tile shape");
+    __shared__ float red[TPP][G * D];
+    __shared__ float qb[G * D];
+
+    const int i = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    SeqInfo s;
+    if (!load_seq(p, b, s)) return;
+    const int nqb = (s.Lq + p.B - 1) / p.B;
+    if (i >= nqb) return;
+    const int t0 = i * p.B;
+    const int n = min(p.B, s.Lq - t0);
+    const int iabs = s.P / p.B + i;
+
+    const int v = threadIdx.x % VPT, tg = threadIdx.x / VPT;
+    float acc[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+    const uint8_t* qrow = Q + (((size_t)(s.q0 + t0) * p.Hq + hk * G) * D) * ELT + (size_t)v * 16;
+    const size_t tok_stride = (size_t)p.Hq * D * ELT;
+    for (int t = tg; t < n; t += TPP) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(qrow + (size_t)t * tok_stride));
+        float f[VEC];
+        unpack16<FP8>(x, f);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += f[e];
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) red[tg][v * VEC + e] = acc[e];
+    __syncthreads();
+    const float inv = 1.f / (float)n;
+    for (int c = threadIdx.x; c < G * D; c += 256) {
+        float sum = 0.f;
+#pragma unroll
+        for (int r = 0; r < TPP; ++r) sum += red[r][c];
+        qb[c] = sum * inv * (FP8 ? p.q_scale[hk * G + c / D] : 1.f);
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int PER_LANE = D / 32;  // 4 (d=128) or 2 (d=64)
+    float qv[G][PER_LANE];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < PER_LANE; ++e) qv[g][e] = qb[g * D + lane * PER_LANE + e];
+    const float scale = rsqrtf((float)D);
+    const float* kb = p.kbar + ((size_t)b * p.Hkv + hk) * p.nkb_max * D + lane * PER_LANE;
+    float* srow = p.scores + (((size_t)b * p.Hq + hk * G) * p.nqb_max + i) * p.nkb_max;
+    const size_t head_stride = (size_t)p.nqb_max * p.nkb_max;
+    for (int j = warp; j <= iabs; j += 8) {
+        float kv[PER_LANE];
+        if constexpr (PER_LANE == 4) {
+            const float4 t = __ldg(reinterpret_cast<const float4*>(kb + (size_t)j * D));
+            kv[0] = t.x; kv[1] = t.y; kv[2] = t.z; kv[3] = t.w;
+        } else {
+            const float2 t = __ldg(reinterpret_cast<const float2*>(kb + (size_t)j * D));
+            kv[0] = t.x; kv[1] = t.y;
+        }
+        float dot[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < PER_LANE; ++e) a = fmaf(qv[g][e], kv[e], a);
+            dot[g] = a;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int g = 0; g < G; ++g) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
+        if (lane < G) {
+            float mine = dot[0];
+#pragma unroll
+            for (int g = 1; g < G; ++g) if (lane == g) mine = dot[g];
+            srow[(size_t)lane * head_stride + j] = mine * scale;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ mask ---
+// One warp per (sequence, query head, query block): row maximum over the
+// causal blocks, then keep j iff s_ij >= max - tau, or j == 0, or j == i_abs.
+// Emits the kept bitmask (all nw words), the ascending kept list and count.
+__global__ void __launch_bounds__(128) mask_kernel(KParams p, float tau) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 4 + warp;
+    const long long nrows = (long long)p.num_seqs * p.Hq * p.nqb_max;
+    if (row >= nrows) return;
+    const int i = (int)(row % p.nqb_max);
+    const int b = (int)(row / ((long long)p.nqb_max * p.Hq));
+    SeqInfo s;
+    if (!load_seq(p, b, s)) return;
+    const int nqb = (s.Lq + p.B - 1) / p.B;
+    if (i >= nqb) return;
+    const int iabs = s.P / p.B + i;
+    const float* S = p.scores + (size_t)row * p.nkb_max;
+    float m = -INFINITY;
+    for (int j = lane; j <= iabs; j += 32) m = fmaxf(m, S[j]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float thr = m - tau;
+    int cnt = 0;
+    uint32_t* bits = p.kept_bits + (size_t)row * p.nw;
+    int32_t* idx = p.kept_idx + (size_t)row * p.nkb_max;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int w = 0; w < p.nw; ++w) {
+        const int j = w * 32 + lane;
+        bool keep = false;
+        if (j <= iabs) keep = (S[j] >= thr) || j == 0 || j == iabs;
+        const uint32_t ball = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) bits[w] = ball;
+        if (keep) idx[cnt + __popc(ball & below)] = j;
+        cnt += __popc(ball);
+    }
+    if (lane == 0) p.kept_cnt[row] = cnt;
+}
+
+// -------------------------------------------------------------- launchers ---
+cudaError_t launch_blockmean(const KParams& p, const void* k, const void* v, cudaStream_t st) {
+    dim3 grid(p.nkb_max, p.Hkv, p.num_seqs);
+    auto K = static_cast<const uint8_t*>(k);
+    auto V = static_cast<const uint8_t*>(v);
+    if (p.fp8) {
+        if (p.d == 128) blockmean_kernel<128, true><<<grid, 128, 0, st>>>(p, K, V);
+        else blockmean_kernel<64, true><<<grid, 128, 0, st>>>(p, K, V);
+    } else {
+        if (p.d == 128) blockmean_kernel<128, false><<<grid, 128, 0, st>>>(p, K, V);
+        else blockmean_kernel<64, false><<<grid, 128, 0, st>>>(p, K, V);
+    }
+    return cudaGetLastError();
+}
+
+template <int D, bool FP8>
+static void score_dispatch_g(const KParams& p, const uint8_t* Q, dim3 grid, cudaStream_t st) {
+    switch (p.G) {
+        case 1: score_kernel<D, FP8, 1><<<grid, 256, 0, st>>>(p, Q); break;
+        case 2: score_kernel<D, FP8, 2><<<grid, 256, 0, st>>>(p, Q); break;
+        case 4: score_kernel<D, FP8, 4><<<grid, 256, 0, st>>>(p, Q); break;
+        default: score_kernel<D, FP8, 8><<<grid, 256, 0, st>>>(p, Q); break;
+    }
+}
+
+cudaError_t launch_score(const KParams& p, const void* q, cudaStream_t st) {
+    dim3 grid(p.nqb_max, p.Hkv, p.num_seqs);
+    auto Q = static_cast<const uint8_t*>(q);
+    if (p.fp8) {
+        if (p.d == 128) score_dispatch_g<128, true>(p, Q, grid, st);
+        else score_dispatch_g<64, true>(p, Q, grid, st);
+    } else {
+        if (p.d == 128) score_dispatch_g<128, false>(p, Q, grid, st);
+        else score_dispatch_g<64, false>(p, Q, grid, st);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mask(const KParams& p, float tau, cudaStream_t st) {
+    const long long rows = (long long)p.num_seqs * p.Hq * p.nqb_max;
+    const unsigned blocks = (unsigned)((rows + 3) / 4);
+    mask_kernel<<<blocks, 128, 0, st>>>(p, tau);
+    return cudaGetLastError();
+}
+
+}  // namespace fp2

@@ -1,0 +1,281 @@
+"""ctypes binding of ``libfp2.so`` (include/fp2.h), with the same names.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are passed by ``data_ptr()``; the stream defaults to
+torch's current stream.  PyTorch is used for device memory and streams.
+There is no fallback: if the library is missing, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp2.so")
+
+FP2_OK = 0
+FP2_ERR_INVALID_ARG = 1
+FP2_ERR_UNSUPPORTED = 2
+FP2_ERR_WORKSPACE = 3
+FP2_ERR_CUDA = 4
+FP2_ERR_TIMEOUT = 5
+FP2_ERR_DEVICE_BOUNDS = 6
+
+FP2_BF16 = 0
+FP2_FP8_E4M3 = 1
+
+
+class Fp2Error(RuntimeError):
+    def __init__(self, status: int, where: str, detail: int = 0):
+        self.status = status
+        self.detail = detail
+        msg = status_string(status) if _LIB is not None else str(status)
+        super().__init__(f"{where}: {msg} (status {status}, detail {detail})")
+
+
+class Params(ctypes.Structure):
+    """Mirror of ``fp2_params``."""
+    _fields_ = [
+        ("num_seqs", ctypes.c_int),
+        ("num_q_heads", ctypes.c_int),
+        ("num_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("total_q", ctypes.c_int),
+        ("total_k", ctypes.c_int),
+        ("page_size", ctypes.c_int),
+        ("max_pages_per_seq", ctypes.c_int),
+        ("num_pages", ctypes.c_int),
+        ("max_seqlen_q", ctypes.c_int),
+        ("max_seqlen_k", ctypes.c_int),
+        ("seqlens_k", ctypes.c_void_p),
+        ("cu_seqlens_k", ctypes.c_void_p),
+        ("q_scale", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p),
+        ("v_scale", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("stream", ctypes.c_void_p),
+    ]
+
+
+class WorkspaceLayout(ctypes.Structure):
+    """Mirror of ``fp2_workspace_layout``."""
+    _fields_ = [
+        ("error_word", ctypes.c_size_t),
+        ("kbar", ctypes.c_size_t),
+        ("vbar", ctypes.c_size_t),
+        ("kbar_op", ctypes.c_size_t),
+        ("vbar_op", ctypes.c_size_t),
+        ("scores", ctypes.c_size_t),
+        ("kept_idx", ctypes.c_size_t),
+        ("kept_cnt", ctypes.c_size_t),
+        ("kept_bits", ctypes.c_size_t),
+        ("total", ctypes.c_size_t),
+        ("nqb_max", ctypes.c_int),
+        ("nkb_max", ctypes.c_int),
+        ("nw", ctypes.c_int),
+    ]
+
+
+_LIB = None
+_VP = ctypes.c_void_p
+_PP = ctypes.POINTER(Params)
+
+# name -> (restype, argtypes); the exported C-ABI
+SIGNATURES = {
+    "fp2_workspace_size": (ctypes.c_size_t, [_PP, ctypes.c_int]),
+    "fp2_get_workspace_layout": (ctypes.c_int, [_PP, ctypes.c_int, ctypes.POINTER(WorkspaceLayout)]),
+    "fp2_prefill": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, ctypes.c_float, ctypes.c_int,
+                                   ctypes.c_int, _VP, _PP]),
+    "fp2_blockmean": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, ctypes.c_int, _PP]),
+    "fp2_score": (ctypes.c_int, [_VP, _VP, ctypes.c_int, ctypes.c_int, _PP]),
+    "fp2_mask": (ctypes.c_int, [_VP, ctypes.c_float, ctypes.c_int, _PP]),
+    "fp2_attn": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int, ctypes.c_int, _VP,
+                                _PP]),
+    "fp2_workspace_init": (ctypes.c_int, [_PP]),
+    "fp2_get_status": (ctypes.c_int, [_PP, ctypes.POINTER(ctypes.c_uint32)]),
+    "fp2_calibrate_tau": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_float, _PP,
+                                         ctypes.POINTER(ctypes.c_float)]),
+    "fp2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "fp2_version": (ctypes.c_char_p, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it was not built (no fallback)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m block_sparse_long_blockmean_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = h
+    return _LIB
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _check(st: int, where: str):
+    if st != FP2_OK:
+        raise Fp2Error(st, where)
+
+
+def status_string(st: int) -> str:
+    return lib().fp2_status_string(st).decode()
+
+
+def version() -> str:
+    return lib().fp2_version().decode()
+
+
+def workspace_size(params: Params, block: int) -> int:
+    return int(lib().fp2_workspace_size(ctypes.byref(params), block))
+
+
+def get_workspace_layout(params: Params, block: int) -> WorkspaceLayout:
+    L = WorkspaceLayout()
+    _check(lib().fp2_get_workspace_layout(ctypes.byref(params), block, ctypes.byref(L)),
+           "fp2_get_workspace_layout")
+    return L
+
+
+def prefill(q, k_cache, v_cache, page_table, cu_seqlens, tau: float, block: int, dtype: int,
+            out, params: Params) -> None:
+    _check(lib().fp2_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                             _ptr(cu_seqlens), float(tau), block, dtype, _ptr(out),
+                             ctypes.byref(params)), "fp2_prefill")
+
+
+def blockmean(k_cache, v_cache, page_table, cu_seqlens, block: int, dtype: int,
+              params: Params) -> None:
+    _check(lib().fp2_blockmean(_ptr(k_cache), _ptr(v_cache), _ptr(page_table), _ptr(cu_seqlens),
+                               block, dtype, ctypes.byref(params)), "fp2_blockmean")
+
+
+def score(q, cu_seqlens, block: int, dtype: int, params: Params) -> None:
+    _check(lib().fp2_score(_ptr(q), _ptr(cu_seqlens), block, dtype, ctypes.byref(params)),
+           "fp2_score")
+
+
+def mask(cu_seqlens, tau: float, block: int, params: Params) -> None:
+    _check(lib().fp2_mask(_ptr(cu_seqlens), float(tau), block, ctypes.byref(params)), "fp2_mask")
+
+
+def attn(q, k_cache, v_cache, page_table, cu_seqlens, kept_bits, block: int, dtype: int, out,
+         params: Params) -> None:
+    _check(lib().fp2_attn(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                          _ptr(cu_seqlens), _ptr(kept_bits), block, dtype, _ptr(out),
+                          ctypes.byref(params)), "fp2_attn")
+
+
+def workspace_init(params: Params) -> None:
+    _check(lib().fp2_workspace_init(ctypes.byref(params)), "fp2_workspace_init")
+
+
+def get_status(params: Params) -> tuple[int, int]:
+    det = ctypes.c_uint32(0)
+    st = lib().fp2_get_status(ctypes.byref(params), ctypes.byref(det))
+    return int(st), int(det.value)
+
+
+def calibrate_tau(cu_seqlens, block: int, target_drop: float, params: Params) -> float:
+    t = ctypes.c_float(0.0)
+    _check(lib().fp2_calibrate_tau(_ptr(cu_seqlens), block, float(target_drop),
+                                   ctypes.byref(params), ctypes.byref(t)), "fp2_calibrate_tau")
+    return float(t.value)
+
+
+# ---------------------------------------------------------------------------
+# convenience: parameters from tensors, a torch-allocated workspace, views of
+# the workspace's intermediates
+# ---------------------------------------------------------------------------
+
+@dataclass
+class Problem:
+    """Device tensors of one call plus its fp2_params (keeps them alive)."""
+    q: object
+    k: object
+    v: object
+    page_table: object
+    cu_seqlens: object
+    out: object
+    block: int
+    dtype: int
+    params: Params
+    workspace: object
+    keep: tuple = ()
+
+    def layout(self) -> WorkspaceLayout:
+        return get_workspace_layout(self.params, self.block)
+
+    def ws_view(self, name: str, torch_dtype, shape):
+        """A tensor view of one workspace region (see WorkspaceLayout)."""
+        import torch
+        L = self.layout()
+        off = getattr(L, name)
+        n = 1
+        for s in shape:
+            n *= s
+        itemsize = torch.empty((), dtype=torch_dtype).element_size()
+        return self.workspace[off: off + n * itemsize].view(torch_dtype).view(*shape)
+
+    def prefill(self, tau: float):
+        prefill(self.q, self.k, self.v, self.page_table, self.cu_seqlens, tau, self.block,
+                self.dtype, self.out, self.params)
+
+    def check(self):
+        st, det = get_status(self.params)
+        if st != FP2_OK:
+            raise Fp2Error(st, "device", det)
+
+
+def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, dtype: int,
+                 max_seqlen_q: int, max_seqlen_k: int, seqlens_k=None, cu_seqlens_k=None,
+                 page_table=None, page_size: int = 0, q_scale=None, k_scale=None,
+                 v_scale=None, out=None, stream=None, workspace=None) -> Problem:
+    """Builds fp2_params for device tensors and allocates the workspace and
+    the bf16 output with torch (allocation only)."""
+    import torch
+    dev = q.device
+    P = Params()
+    P.num_seqs = int(cu_seqlens.numel() - 1)
+    P.num_q_heads, P.num_kv_heads, P.head_dim = Hq, Hkv, d
+    P.total_q = int(q.shape[0])
+    if page_table is None:
+        P.total_k = int(k.shape[0])
+    else:
+        P.total_k = 0
+        P.page_size = page_size
+        P.max_pages_per_seq = int(page_table.shape[1])
+        P.num_pages = int(k.shape[0])
+    P.max_seqlen_q, P.max_seqlen_k = int(max_seqlen_q), int(max_seqlen_k)
+    P.seqlens_k = _ptr(seqlens_k)
+    P.cu_seqlens_k = _ptr(cu_seqlens_k)
+    P.q_scale, P.k_scale, P.v_scale = _ptr(q_scale), _ptr(k_scale), _ptr(v_scale)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    P.stream = stream
+    nbytes = workspace_size(P, block)
+    if nbytes == 0:
+        raise Fp2Error(FP2_ERR_INVALID_ARG, "fp2_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    P.workspace = workspace.data_ptr()
+    P.workspace_bytes = workspace.numel()
+    workspace_init(P)
+    if out is None:
+        out = torch.empty((q.shape[0], Hq, d), dtype=torch.bfloat16, device=dev)
+    keep = (seqlens_k, cu_seqlens_k, q_scale, k_scale, v_scale)
+    return Problem(q, k, v, page_table, cu_seqlens, out, block, dtype, P, workspace, keep)

@@ -1,0 +1,184 @@
+/*
+ * fp2.h -- C ABI of the B200 (sm_100a) block-sparse causal prefill attention
+ * with block-mean correction (FlashPrefill V2).
+ *
+ * The method (FlashPrefill V2 abstract, chatpaper.ai card, English abstract;
+ * popular explainer, papers.ananclaw.com, sections 2.1-2.3):
+ *   1. block means kbar_j, vbar_j of K and V per KV head       (fp2_blockmean)
+ *   2. pooled query blocks scored against every causal key
+ *      block ("instantaneous pattern discovery")                (fp2_score)
+ *   3. max-based dynamic threshold: keep j iff
+ *      s_ij >= max_j' s_ij' - tau; block 0 and the diagonal
+ *      block are always kept                                    (fp2_mask)
+ *   4. online-softmax attention over the kept blocks, GQA heads
+ *      packed so a K/V tile is loaded once per group (PackGQA),
+ *      plus the mean correction: every dropped block j enters
+ *      the same softmax as one pseudo-token with weight
+ *      n_j * exp(q.kbar_j / sqrt(d)) and value vbar_j          (fp2_attn)
+ * fp2_prefill runs the four in order on one stream.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument is a DEVICE pointer unless its comment says host.
+ *    The caller owns every buffer; the library never allocates, frees or
+ *    synchronises on these calls: all work is enqueued on params->stream
+ *    (a cudaStream_t; NULL = the legacy default stream) and the call returns
+ *    before it runs.
+ *  - q and out are [total_q, Hq, d], row-major, sequences packed by
+ *    cu_seqlens (int32 [num_seqs+1], device, cu_seqlens[0] = 0).
+ *  - Contiguous K/V (page_table == NULL): k_cache, v_cache are
+ *    [total_k, Hkv, d] packed by params->cu_seqlens_k (or by cu_seqlens when
+ *    that is NULL).  Paged K/V: [num_pages, page_size, Hkv, d] with
+ *    page_table int32 [num_seqs, max_pages_per_seq] of physical page ids.
+ *  - Sequence b has Lq = cu_seqlens[b+1]-cu_seqlens[b] new tokens and
+ *    Lk = seqlens_k[b] (or Lq when seqlens_k is NULL) keys; query t sits at
+ *    absolute position Lk - Lq + t.  Lk - Lq (the resident prefix) must be a
+ *    multiple of the block size.
+ *  - dtype FP2_BF16: q/k/v are bf16.  FP2_FP8_E4M3: q/k/v are e4m3 with
+ *    per-head dequantisation scales (x = e4m3 * scale), params->q_scale [Hq],
+ *    k_scale [Hkv], v_scale [Hkv] (fp32, device).  out is always bf16.
+ *  - Base pointers of q, k_cache, v_cache and out must be 16-byte aligned.
+ *  - Supported: head_dim 64 or 128 (FP8: 128), block 64 or 128,
+ *    G = Hq/Hkv in {1,2,4,8} with 128/G <= block, page_size a power of two
+ *    in [16, 256] that divides the block or is divided by it.
+ *
+ * Errors: argument errors are returned synchronously before any launch.
+ * CUDA launch errors return FP2_ERR_CUDA.  Problems only the device can see
+ * (a prefix that is not a multiple of the block, Lk < Lq, a length above
+ * max_seqlen_*, a page id outside [0, num_pages), a bounded wait that ran
+ * out) set an error word in the workspace and make the affected blocks skip
+ * their work; fp2_get_status reads it.  Nothing prints, nothing throws.
+ */
+#ifndef FP2_H
+#define FP2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP2_OK = 0,
+    FP2_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent shapes */
+    FP2_ERR_UNSUPPORTED = 2,   /* valid but outside the supported set above */
+    FP2_ERR_WORKSPACE = 3,     /* workspace missing or smaller than fp2_workspace_size */
+    FP2_ERR_CUDA = 4,          /* a CUDA call failed */
+    FP2_ERR_TIMEOUT = 5,       /* device: a bounded pipeline wait ran out */
+    FP2_ERR_DEVICE_BOUNDS = 6  /* device: an index (page id, length) out of range */
+} fp2_status;
+
+typedef enum { FP2_BF16 = 0, FP2_FP8_E4M3 = 1 } fp2_dtype;
+
+typedef struct fp2_params {
+    int num_seqs;              /* >= 1 */
+    int num_q_heads;           /* Hq */
+    int num_kv_heads;          /* Hkv, divides Hq */
+    int head_dim;              /* d */
+    int total_q;               /* rows of q and out */
+    int total_k;               /* contiguous K/V: rows of k_cache/v_cache; paged: 0 */
+    int page_size;             /* paged only: tokens per page */
+    int max_pages_per_seq;     /* paged only: row stride of page_table */
+    int num_pages;             /* paged only: pages in k_cache/v_cache */
+    int max_seqlen_q;          /* >= every Lq; sizes the workspace */
+    int max_seqlen_k;          /* >= every Lk; sizes the workspace */
+    const int32_t* seqlens_k;  /* device [num_seqs] or NULL (Lk = Lq) */
+    const int32_t* cu_seqlens_k; /* device [num_seqs+1], contiguous K/V only, or NULL */
+    const float* q_scale;      /* FP8 only, device [Hq] */
+    const float* k_scale;      /* FP8 only, device [Hkv] */
+    const float* v_scale;      /* FP8 only, device [Hkv] */
+    void* workspace;           /* device, fp2_workspace_size() bytes, 256-byte aligned */
+    size_t workspace_bytes;
+    void* stream;              /* cudaStream_t */
+} fp2_params;
+
+/* Offsets (bytes from params->workspace) of the intermediates, for callers
+ * that read them (parity checks, exported masks).  Per-sequence regions are
+ * padded to nqb_max = ceil(max_seqlen_q/B) query blocks and
+ * nkb_max = ceil(max_seqlen_k/B) key blocks; nw = ceil(nkb_max/32). */
+typedef struct fp2_workspace_layout {
+    size_t error_word;  /* uint32 [4]: first error code, detail */
+    size_t kbar;        /* fp32 [num_seqs][Hkv][nkb_max][d]: dequantised key block means */
+    size_t vbar;        /* fp32 [num_seqs][Hkv][nkb_max][d] */
+    size_t kbar_op;     /* bf16|e4m3 [num_seqs][Hkv][nkb_max][d]: means as MMA operands */
+    size_t vbar_op;     /* (FP8: in the units of k_scale / v_scale) */
+    size_t scores;      /* fp32 [num_seqs][Hq][nqb_max][nkb_max], j <= i_abs written */
+    size_t kept_idx;    /* int32 [num_seqs][Hq][nqb_max][nkb_max], ascending kept j */
+    size_t kept_cnt;    /* int32 [num_seqs][Hq][nqb_max] */
+    size_t kept_bits;   /* uint32 [num_seqs][Hq][nqb_max][nw], bit j = block j kept */
+    size_t total;       /* bytes needed */
+    int nqb_max, nkb_max, nw;
+} fp2_workspace_layout;
+
+/* Workspace bytes for these params and block size (0 on invalid params). */
+size_t fp2_workspace_size(const fp2_params* params, int block);
+
+/* Fills *layout; FP2_ERR_INVALID_ARG on invalid params. */
+fp2_status fp2_get_workspace_layout(const fp2_params* params, int block,
+                                    fp2_workspace_layout* layout);
+
+/* The whole path: blockmean -> score -> mask -> attn.  tau >= 0 or +inf is
+ * the usual range (any non-NaN value is accepted; tau = +inf keeps every
+ * block and gives exact causal attention).  out: bf16 [total_q, Hq, d]. */
+fp2_status fp2_prefill(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* page_table, const int32_t* cu_seqlens,
+                       float tau, int block, fp2_dtype dtype, void* out,
+                       const fp2_params* params);
+
+/* Step 1 (explainer section 2.1, the mean of the dropped tokens): block means
+ * of K and V into the workspace (kbar, vbar, kbar_op, vbar_op); key blocks
+ * beyond a sequence's end are written as zeros. */
+fp2_status fp2_blockmean(const void* k_cache, const void* v_cache, const int32_t* page_table,
+                         const int32_t* cu_seqlens, int block, fp2_dtype dtype,
+                         const fp2_params* params);
+
+/* Step 2 (abstract: instantaneous pattern discovery): pools each query block
+ * (mean of its valid rows) and writes s_ij = qbar_i . kbar_j / sqrt(d) for
+ * every causal j into the workspace scores.  Needs step 1. */
+fp2_status fp2_score(const void* q, const int32_t* cu_seqlens, int block, fp2_dtype dtype,
+                     const fp2_params* params);
+
+/* Step 3 (abstract: max-based dynamic thresholding): writes kept_idx,
+ * kept_cnt and kept_bits into the workspace.  Needs step 2. */
+fp2_status fp2_mask(const int32_t* cu_seqlens, float tau, int block, const fp2_params* params);
+
+/* Step 4 (abstract: sparse operator with PackGQA, warp specialisation and
+ * pipelining; the mean correction term): tcgen05/TMEM attention over the
+ * blocks set in kept_bits (uint32 [num_seqs][Hq][nqb_max][nw], the layout of
+ * the workspace's kept_bits; pass NULL to use the workspace's own), with the
+ * block-mean pseudo-tokens for every causal block that is not set.  Needs
+ * step 1 (the means).  Bits for j > i_abs are ignored; block 0 and the
+ * diagonal are treated as set whatever the bits say. */
+fp2_status fp2_attn(const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* page_table, const int32_t* cu_seqlens,
+                    const uint32_t* kept_bits, int block, fp2_dtype dtype, void* out,
+                    const fp2_params* params);
+
+/* Zeroes the workspace's error word (asynchronously, on params->stream).
+ * Call it once on a new workspace before the first call that uses it; after
+ * that fp2_get_status keeps it clear. */
+fp2_status fp2_workspace_init(const fp2_params* params);
+
+/* Synchronises params->stream, returns the first device-side error recorded
+ * in the workspace since the last call (FP2_OK if none) and clears it.
+ * detail (host, may be NULL) receives the error's detail word. */
+fp2_status fp2_get_status(const fp2_params* params, uint32_t* detail);
+
+/* Host utility, not on the hot path (synchronises): the tau at which the
+ * scores in the workspace (after fp2_score) drop target_drop of all causal
+ * block pairs (forced blocks counted as kept): the midpoint of the two
+ * adjacent margins max_j' s_ij' - s_ij at that quantile.  *tau_out is host. */
+fp2_status fp2_calibrate_tau(const int32_t* cu_seqlens, int block, float target_drop,
+                             const fp2_params* params, float* tau_out);
+
+/* Static string naming a status code. */
+const char* fp2_status_string(fp2_status status);
+
+/* Library version, "major.minor.patch". */
+const char* fp2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP2_H */

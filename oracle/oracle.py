@@ -243,3 +243,29 @@ def tau_for_drop(S_list, prefix_blocks_list, target: float, guard: float = 0.0):
         raise ValueError("no gap wide enough for the guard")
     best = ok[np.argmin(np.abs(ok - (k - 1)))]
     return 0.5 * (float(a[best]) + float(a[best + 1]))
+
+
+def attn_query_block(Qblk, K, V, kbar, vbar, cnt, keep_i, B: int, iabs: int, heads=None,
+                     mutant: int = 0):
+    """Corrected attention of ONE query block at absolute block index ``iabs``.
+
+    ``Qblk`` [n, Hq, d] holds the block's rows, ``keep_i`` [Hq, >= iabs+1] its
+    mask row.  Calls ``attn_rows`` on the causal window: keys ``[0, iabs*B+n)``
+    (later keys never reach these rows) with the block as the whole query
+    side, so that prefix = iabs*B puts every row at its true position.  No
+    arithmetic of its own; it lets a long sequence be checked block by block
+    without an fp64 copy of all of Q.  Returns [n * len(heads), d] ordered
+    (row, head)."""
+    Qblk = _f64(Qblk)
+    n, Hq, d = Qblk.shape
+    Lk = iabs * B + n
+    nkb = iabs + 1
+    if heads is None:
+        heads = np.arange(Hq, dtype=np.int32)
+    heads = np.asarray(heads, dtype=np.int32)
+    rows = np.repeat(np.arange(n, dtype=np.int32), heads.size)
+    hh = np.tile(heads, n)
+    keep = np.ascontiguousarray(np.asarray(keep_i)[:, None, :nkb], dtype=np.uint8)
+    return attn_rows(Qblk, np.asarray(K)[:Lk], np.asarray(V)[:Lk], np.asarray(kbar)[:, :nkb],
+                     np.asarray(vbar)[:, :nkb], np.asarray(cnt)[:nkb], keep, B, rows, hh,
+                     mutant=mutant)
