@@ -38,6 +38,9 @@ def parse():
     ap.add_argument("--impl", default="fp2", choices=["fp2", "reference"])
     ap.add_argument("--dtype", default="both", choices=["bf16", "fp8", "both"])
     ap.add_argument("--drop", type=float, default=DROP)
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[2, 3],
+                    help="3 = the 128K layer (the metric's workload); 2 = the 32K layer, a "
+                         "smaller case for profiler captures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -150,7 +153,7 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
     from block_sparse_long_blockmean_b200 import fp2, synth
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    shape = synth.workload(WORKLOAD_ID, dtype_name)
+    shape = synth.workload(args.workload, dtype_name)
     t0 = time.time()
     inp = synth.make_inputs(shape)
     gen_s = time.time() - t0
@@ -316,7 +319,7 @@ def reference_arm(args):
     sample of the same layer (one query block x 4 heads), scaled to ms/layer."""
     from block_sparse_long_blockmean_b200 import synth
     from oracle import oracle as O
-    shape = synth.workload(WORKLOAD_ID, "bf16")
+    shape = synth.workload(args.workload, "bf16")
     inp = synth.make_inputs(shape)
     s = shape
     B = s.B
@@ -349,7 +352,7 @@ def reference_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": synth.WORKLOAD_NAMES[WORKLOAD_ID], "drop": args.drop},
+            "config": {"workload": synth.WORKLOAD_NAMES[args.workload], "drop": args.drop},
             "cpu_baseline": {"value": ms, "unit": "ms/layer", "cores": O.num_threads(),
                              "kind": "oracle",
                              "sample": "per step: corrected attention of 4 heads x 1 random "
@@ -416,7 +419,8 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": main_dt,
         "data": "synthetic",
-        "config": {"workload": synth.WORKLOAD_NAMES[WORKLOAD_ID], "seq_len": 131072,
+        "config": {"workload": synth.WORKLOAD_NAMES[args.workload],
+                   "seq_len": synth.workload(args.workload).lens_q[0],
                    "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128, "block": 128,
                    "target_drop": args.drop, "layout": "contiguous K/V",
                    "l2": "inputs (1.6 GB) larger than L2; no flush",
