@@ -88,6 +88,8 @@ SIGNATURES = {
     "fp2_get_workspace_layout": (ctypes.c_int, [_PP, ctypes.c_int, ctypes.POINTER(WorkspaceLayout)]),
     "fp2_prefill": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, ctypes.c_float, ctypes.c_int,
                                    ctypes.c_int, _VP, _PP]),
+    "fp2_prefill_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, ctypes.c_float, ctypes.c_int,
+                                           ctypes.c_int, _VP, _PP]),
     "fp2_blockmean": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, ctypes.c_int, _PP]),
     "fp2_score": (ctypes.c_int, [_VP, _VP, ctypes.c_int, ctypes.c_int, _PP]),
     "fp2_mask": (ctypes.c_int, [_VP, ctypes.c_float, ctypes.c_int, _PP]),
@@ -156,6 +158,14 @@ def prefill(q, k_cache, v_cache, page_table, cu_seqlens, tau: float, block: int,
     _check(lib().fp2_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
                              _ptr(cu_seqlens), float(tau), block, dtype, _ptr(out),
                              ctypes.byref(params)), "fp2_prefill")
+
+
+def prefill_noalloc(q, k_cache, v_cache, page_table, cu_seqlens, tau: float, block: int,
+                    dtype: int, out, params: Params) -> None:
+    """fp2_prefill with library-owned scratch (params.workspace is ignored)."""
+    _check(lib().fp2_prefill_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                                     _ptr(cu_seqlens), float(tau), block, dtype, _ptr(out),
+                                     ctypes.byref(params)), "fp2_prefill_noalloc")
 
 
 def blockmean(k_cache, v_cache, page_table, cu_seqlens, block: int, dtype: int,

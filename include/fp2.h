@@ -172,6 +172,35 @@ fp2_status fp2_get_status(const fp2_params* params, uint32_t* detail);
 fp2_status fp2_calibrate_tau(const int32_t* cu_seqlens, int block, float target_drop,
                              const fp2_params* params, float* tau_out);
 
+/* Bytes of the library-owned device scratch used by fp2_prefill_noalloc. */
+#define FP2_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* fp2_prefill for callers that cannot allocate device memory.  The paper has
+ * no counterpart: this is a packaging variant, not a step of the method.
+ * Plugin-style hosts that hand a kernel only its inputs and outputs, and
+ * serving runtimes that reserve all device memory up front (so that a
+ * cudaMalloc on the request path would fail or stall the device), cannot
+ * supply the workspace fp2_prefill needs.  This call takes the same
+ * arguments, ignores params->workspace / params->workspace_bytes, and keeps
+ * its scratch in a library-owned device array of FP2_NOALLOC_SCRATCH_BYTES
+ * (every GPU that loads the library holds it until the process exits).  It
+ * allocates nothing.
+ *  - A problem whose fp2_workspace_size() exceeds FP2_NOALLOC_SCRATCH_BYTES
+ *    (e.g. one 32K-token sequence with 32 query heads fits; 128K does not) is
+ *    rejected with FP2_ERR_WORKSPACE before anything is queued.
+ *  - The first call on a device looks up the array's device address (a
+ *    synchronous runtime query, once per device); make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array and leaves its contents behind; calls
+ *    whose work overlaps on the GPU (other streams, other host threads) race
+ *    on it, so the caller must serialise them.
+ *  - The array's error word is cleared at the start of each call; device-side
+ *    errors of this call cannot be read with fp2_get_status. */
+fp2_status fp2_prefill_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* page_table, const int32_t* cu_seqlens,
+                               float tau, int block, fp2_dtype dtype, void* out,
+                               const fp2_params* params);
+
 /* Static string naming a status code. */
 const char* fp2_status_string(fp2_status status);
 

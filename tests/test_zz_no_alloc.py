@@ -1,0 +1,55 @@
+"""fp2_prefill_noalloc -- the prefill for callers that cannot allocate device
+memory (plugin-style hosts that pass a kernel only its inputs and outputs,
+runtimes that reserve all device memory up front) -- checked through the C ABI
+against fp2_prefill on the same inputs, on two calls in a row.  This file is
+collected last on purpose: it must pass alone in a fresh process and after
+every other test."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_blockmean_b200 import fp2, synth
+from oracle import oracle as O
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype,page", [("bf16", 64), ("fp8", 0)])
+def test_noalloc_matches_prefill_on_two_calls(dtype, page):
+    shape = H.small_shape([700, 300], lens_k=[256 + 700, 300], Hq=8, Hkv=2, dtype=dtype,
+                          page_size=page if page else 0, seed=23)
+    if page == 0:  # contiguous K/V cannot carry a prefix
+        shape.lens_k = list(shape.lens_q)
+    inp = synth.make_inputs(shape)
+    orc = H.oracle_scores(inp)
+    tau = H.pick_tau(orc, 0.6)
+    pr = H.problem(inp)
+    pr.prefill(tau)
+    pr.check()
+    ref = pr.out.double().cpu().numpy()
+    lib = fp2.lib()
+    for call in range(2):
+        out = torch.full_like(pr.out, float("nan"))
+        st = lib.fp2_prefill_noalloc(pr.q.data_ptr(), pr.k.data_ptr(), pr.v.data_ptr(),
+                                     pr.page_table.data_ptr() if pr.page_table is not None else None,
+                                     pr.cu_seqlens.data_ptr(), ctypes.c_float(tau), shape.B,
+                                     pr.dtype, out.data_ptr(), ctypes.byref(pr.params))
+        assert st == fp2.FP2_OK, fp2.status_string(st)
+        torch.cuda.synchronize()
+        got = out.double().cpu().numpy()
+        assert np.isfinite(got).all(), f"call {call}"
+        H.assert_close(got, ref, dtype == "fp8", f"call {call}")
+
+
+def test_noalloc_rejects_problems_above_its_scratch():
+    P = fp2.Params()
+    P.num_seqs, P.num_q_heads, P.num_kv_heads, P.head_dim = 1, 32, 8, 128
+    P.total_q = P.total_k = P.max_seqlen_q = P.max_seqlen_k = 131072
+    assert fp2.workspace_size(P, 128) > 32 * 1024 * 1024
+    fake = 1 << 20
+    st = fp2.lib().fp2_prefill_noalloc(fake, fake, fake, None, fake, ctypes.c_float(1.0), 128,
+                                       fp2.FP2_BF16, fake, ctypes.byref(P))
+    assert st == fp2.FP2_ERR_WORKSPACE
