@@ -13,7 +13,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libfp2.so")
-SOURCES = ["fp2_api.cu", "fp2_stages.cu", "fp2_attn.cu", "fp2_noalloc.cu"]
+SOURCES = ["fp2_api.cu", "fp2_stages.cu", "fp2_attn.cu", "fp2_attn_pair.cu", "fp2_noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,

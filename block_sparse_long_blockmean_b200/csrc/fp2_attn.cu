@@ -30,15 +30,11 @@
 //               (bf16 | e4m3) to shared memory in the 128-byte swizzle
 //               layout, and at the end normalises O and stores bf16 rows.
 // TMEM: S0 cols [0,128), S1 [128,256), O [256,256+d).
-#include <cuda_bf16.h>
-#include <cuda_fp8.h>
+#include <cstdlib>
 
-#include "fp2_seq.cuh"
+#include "fp2_attn_common.cuh"
 
 namespace fp2 {
-
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
-constexpr float kRescaleLog2 = 8.0f;              // lazy-rescale threshold (x256)
 
 template <int D, int BLK, bool FP8>
 struct AttnCfg {
@@ -61,10 +57,6 @@ struct AttnCfg {
     static constexpr int OFF_ITEMS = OFF_MISC + 64;
     static_assert(NCH >= 1 && PCH >= 1, "tile shape");
     static_assert(D % 32 == 0 && BLK % 32 == 0, "tile shape");
-};
-
-struct AttnMaps {
-    CUtensorMap q, k, v, kb, vb;
 };
 
 // barrier slots
@@ -121,61 +113,11 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         tmem_alloc(&misc[0], 512);
         tmem_relinquish();
     }
-    // per-head kept bits of this query block (forced blocks set, j > iabs cleared)
-    const uint32_t* kb_src = kept_bits + (((size_t)b * p.Hq + (size_t)hk * G) * p.nqb_max + i) * p.nw;
-    for (int x = threadIdx.x; x < G * nw_c; x += blockDim.x) {
-        const int g = x / nw_c, w = x % nw_c;
-        uint32_t word = kb_src[(size_t)g * p.nqb_max * p.nw + w];
-        if (w == 0) word |= 1u;
-        if (w == (iabs >> 5)) {
-            word |= 1u << (iabs & 31);
-            const int hi = iabs & 31;
-            if (hi < 31) word &= (2u << hi) - 1u;
-        }
-        sbits[x] = word;
-    }
+    load_kept_bits(p, kept_bits, b, hk, i, iabs, nw_c, sbits);
     __syncthreads();
-    // item list: union of kept blocks (ascending), then mean tiles with a drop
     if (warp == 0) {
-        int base = 0;
-        for (int w0 = 0; w0 < nw_c; w0 += 32) {
-            const int w = w0 + lane;
-            uint32_t u = 0;
-            if (w < nw_c)
-                for (int g = 0; g < G; ++g) u |= sbits[g * nw_c + w];
-            const int c = __popc(u);
-            int incl = c;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            int pos = base + incl - c;
-            while (u) {
-                const int bit = __ffs(u) - 1;
-                u &= u - 1;
-                items[pos++] = w * 32 + bit;
-            }
-            base += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        // virtual tiles: tile t covers mean rows [t*BLK, t*BLK+BLK) of blocks < iabs
-        const int nvt = (iabs + BLK - 1) / BLK;
-        for (int t = 0; t < nvt; ++t) {
-            const int lo = t * BLK, hi = min(iabs, (t + 1) * BLK);  // blocks [lo, hi)
-            const int w_lo = lo >> 5, nwt = ((hi + 31) >> 5) - w_lo;
-            bool any = false;
-            for (int x = lane; x < G * nwt; x += 32) {
-                const int g = x / nwt, w = w_lo + x % nwt;
-                uint32_t m = ~sbits[g * nw_c + w];
-                const int top = hi - w * 32;  // > 0
-                if (top < 32) m &= (1u << top) - 1u;
-                any |= (m != 0u);
-            }
-            any = __any_sync(0xffffffffu, any);
-            if (lane == 0 && any) items[base] = -(t + 1);
-            if (any) ++base;
-        }
-        if (lane == 0) misc[2] = (uint32_t)base;
+        const int n = build_items<BLK>(G, iabs, nw_c, sbits, items);
+        if (lane == 0) misc[2] = (uint32_t)n;
     }
     tc_fence_before();
     __syncthreads();
@@ -196,7 +138,6 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             for (int c = 0; c < C::NCH; ++c)
                 tma_load_3d(q_s + c * (128 * 128), &maps.q, &bars[B_Q_FULL], c * C::CH, hk * G,
                             s.q0 + t_begin);
-            const int R = p.paged ? min(p.page_size, BLK) : BLK;
             int issued = 0;
             for (int n = 0; n < n_items; ++n) {
                 const int st = n & 1;
@@ -205,59 +146,10 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                     set_error(p.err, kErrTimeout, kDetWaitBase + 0);
                     break;
                 }
-                const uint32_t k_s = sbase + C::OFF_K + st * C::KV_BYTES;
-                const uint32_t v_s = sbase + C::OFF_V + st * C::KV_BYTES;
-                const int item = items[n];
-                if (item >= 0) {
-                    const int j = item;
-                    if (!p.paged) {
-                        mbar_arrive_expect_tx(&bars[B_KV_FULL + st], 2 * C::KV_BYTES);
-                        for (int c = 0; c < C::NCH; ++c) {
-                            tma_load_3d(k_s + c * BLK * 128, &maps.k, &bars[B_KV_FULL + st],
-                                        c * C::CH, hk, s.k0 + j * BLK);
-                            tma_load_3d(v_s + c * BLK * 128, &maps.v, &bars[B_KV_FULL + st],
-                                        c * C::CH, hk, s.k0 + j * BLK);
-                        }
-                    } else {
-                        // one box per page of the block that holds keys
-                        int nbox = 0;
-                        int pages[BLK / 16];
-                        for (int sb = 0; sb < BLK / R; ++sb) {
-                            const int tok = j * BLK + sb * R;
-                            int pg = -1;
-                            if (tok < s.Lk) {
-                                pg = p.page_table[(size_t)b * p.max_pages + tok / p.page_size];
-                                if (pg < 0 || pg >= p.num_pages) {
-                                    set_error(p.err, kErrBounds, kDetPage);
-                                    pg = -1;
-                                }
-                            }
-                            pages[sb] = pg;
-                            nbox += (pg >= 0);
-                        }
-                        mbar_arrive_expect_tx(&bars[B_KV_FULL + st],
-                                              (uint32_t)(2 * nbox * C::NCH * R * 128));
-                        for (int sb = 0; sb < BLK / R; ++sb) {
-                            if (pages[sb] < 0) continue;
-                            const int off = (j * BLK + sb * R) % p.page_size;
-                            for (int c = 0; c < C::NCH; ++c) {
-                                tma_load_4d(k_s + c * BLK * 128 + sb * R * 128, &maps.k,
-                                            &bars[B_KV_FULL + st], c * C::CH, hk, off, pages[sb]);
-                                tma_load_4d(v_s + c * BLK * 128 + sb * R * 128, &maps.v,
-                                            &bars[B_KV_FULL + st], c * C::CH, hk, off, pages[sb]);
-                            }
-                        }
-                    }
-                } else {
-                    const int t = -item - 1;
-                    mbar_arrive_expect_tx(&bars[B_KV_FULL + st], 2 * C::KV_BYTES);
-                    for (int c = 0; c < C::NCH; ++c) {
-                        tma_load_3d(k_s + c * BLK * 128, &maps.kb, &bars[B_KV_FULL + st],
-                                    c * C::CH, t * BLK, b * p.Hkv + hk);
-                        tma_load_3d(v_s + c * BLK * 128, &maps.vb, &bars[B_KV_FULL + st],
-                                    c * C::CH, t * BLK, b * p.Hkv + hk);
-                    }
-                }
+                issue_item_loads<D, BLK, FP8>(p, maps, s, b, hk, items[n],
+                                              sbase + C::OFF_K + st * C::KV_BYTES,
+                                              sbase + C::OFF_V + st * C::KV_BYTES,
+                                              &bars[B_KV_FULL + st]);
                 ++issued;
             }
             // never leave with copies in flight: wait (bounded) for the loads
@@ -461,15 +353,9 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             // a partial last key block: zero the V rows past the sequence end
             // (they may hold stale page contents; P is zero there, but 0 * NaN
             // would not be)
-            if (item >= 0 && item * BLK + BLK > s.Lk) {
-                const int nvalid = max(0, s.Lk - item * BLK);
-                uint8_t* v_tile = smem + C::OFF_V + st * C::KV_BYTES;
-                const int units = (BLK - nvalid) * 8;  // 16-byte units per chunk
-                for (int c = 0; c < C::NCH; ++c)
-                    for (int x16 = r; x16 < units; x16 += 128)
-                        *reinterpret_cast<uint4*>(v_tile + c * BLK * 128 + nvalid * 128 + x16 * 16) =
-                            make_uint4(0, 0, 0, 0);
-            }
+            if (item >= 0 && item * BLK + BLK > s.Lk)
+                zero_v_tail<BLK, C::NCH>(smem + C::OFF_V + st * C::KV_BYTES,
+                                         max(0, s.Lk - item * BLK), r, 128);
             if (__any_sync(0xffffffffu, rescale && n >= 1)) {
                 const float a = (rescale && n >= 1) ? alpha : 1.f;
 #pragma unroll
@@ -558,43 +444,51 @@ static bool encode(CUtensorMap* m, bool fp8, int rank, const void* base, const c
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int BLK, bool FP8>
-static cudaError_t launch_attn_t(const KParams& p, const void* q, const void* k, const void* v,
-                                 const uint32_t* kept_bits, void* out, cudaStream_t st) {
-    using C = AttnCfg<D, BLK, FP8>;
-    const cuuint64_t E = FP8 ? 1 : 2;
-    AttnMaps maps;
-    const int TOK = 128 / p.G;
+bool make_attn_maps(const KParams& p, const void* q, const void* k, const void* v, int D,
+                    int BLK, int TOK, AttnMaps* maps) {
+    const bool fp8 = p.fp8 != 0;
+    const cuuint64_t E = fp8 ? 1 : 2;
+    const cuuint32_t CH = fp8 ? 128 : 64;
     {
         cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p.Hq, (cuuint64_t)p.total_q};
         cuuint64_t str[2] = {D * E, (cuuint64_t)p.Hq * D * E};
-        cuuint32_t box[3] = {(cuuint32_t)C::CH, (cuuint32_t)p.G, (cuuint32_t)TOK};
-        if (!encode(&maps.q, FP8, 3, q, dims, str, box)) return cudaErrorInvalidValue;
+        cuuint32_t box[3] = {CH, (cuuint32_t)p.G, (cuuint32_t)TOK};
+        if (!encode(&maps->q, fp8, 3, q, dims, str, box)) return false;
     }
     if (!p.paged) {
         cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p.Hkv, (cuuint64_t)p.total_k};
         cuuint64_t str[2] = {D * E, (cuuint64_t)p.Hkv * D * E};
-        cuuint32_t box[3] = {(cuuint32_t)C::CH, 1, (cuuint32_t)BLK};
-        if (!encode(&maps.k, FP8, 3, k, dims, str, box)) return cudaErrorInvalidValue;
-        if (!encode(&maps.v, FP8, 3, v, dims, str, box)) return cudaErrorInvalidValue;
+        cuuint32_t box[3] = {CH, 1, (cuuint32_t)BLK};
+        if (!encode(&maps->k, fp8, 3, k, dims, str, box)) return false;
+        if (!encode(&maps->v, fp8, 3, v, dims, str, box)) return false;
     } else {
         const int R = p.page_size < BLK ? p.page_size : BLK;
         cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)p.Hkv, (cuuint64_t)p.page_size,
                               (cuuint64_t)p.num_pages};
         cuuint64_t str[3] = {D * E, (cuuint64_t)p.Hkv * D * E,
                              (cuuint64_t)p.page_size * p.Hkv * D * E};
-        cuuint32_t box[4] = {(cuuint32_t)C::CH, 1, (cuuint32_t)R, 1};
-        if (!encode(&maps.k, FP8, 4, k, dims, str, box)) return cudaErrorInvalidValue;
-        if (!encode(&maps.v, FP8, 4, v, dims, str, box)) return cudaErrorInvalidValue;
+        cuuint32_t box[4] = {CH, 1, (cuuint32_t)R, 1};
+        if (!encode(&maps->k, fp8, 4, k, dims, str, box)) return false;
+        if (!encode(&maps->v, fp8, 4, v, dims, str, box)) return false;
     }
     {
         cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p.nkb_max,
                               (cuuint64_t)p.num_seqs * p.Hkv};
         cuuint64_t str[2] = {D * E, (cuuint64_t)p.nkb_max * D * E};
-        cuuint32_t box[3] = {(cuuint32_t)C::CH, (cuuint32_t)BLK, 1};
-        if (!encode(&maps.kb, FP8, 3, p.kbar_op, dims, str, box)) return cudaErrorInvalidValue;
-        if (!encode(&maps.vb, FP8, 3, p.vbar_op, dims, str, box)) return cudaErrorInvalidValue;
+        cuuint32_t box[3] = {CH, (cuuint32_t)BLK, 1};
+        if (!encode(&maps->kb, fp8, 3, p.kbar_op, dims, str, box)) return false;
+        if (!encode(&maps->vb, fp8, 3, p.vbar_op, dims, str, box)) return false;
     }
+    return true;
+}
+
+template <int D, int BLK, bool FP8>
+static cudaError_t launch_attn_t(const KParams& p, const void* q, const void* k, const void* v,
+                                 const uint32_t* kept_bits, void* out, cudaStream_t st) {
+    using C = AttnCfg<D, BLK, FP8>;
+    AttnMaps maps;
+    const int TOK = 128 / p.G;
+    if (!make_attn_maps(p, q, k, v, D, BLK, TOK, &maps)) return cudaErrorInvalidValue;
     const int items_cap = p.nkb_max + (p.nkb_max + BLK - 1) / BLK + 2;
     const int nw_c_max = p.nkb_max / 32 + 1;
     size_t smem = 1024 + C::OFF_ITEMS + (size_t)items_cap * 4 + (size_t)p.G * nw_c_max * 4;
@@ -612,8 +506,15 @@ static cudaError_t launch_attn_t(const KParams& p, const void* q, const void* k,
     return cudaGetLastError();
 }
 
+cudaError_t launch_attn_pair(const KParams& p, const void* q, const void* k, const void* v,
+                             const uint32_t* kept_bits, void* out, cudaStream_t st);
+
+// Query blocks of at least 256 packed rows (G * block >= 256) go to the
+// two-tile kernel; smaller ones to the single-tile kernel above.
 cudaError_t launch_attn(const KParams& p, const void* q, const void* k, const void* v,
                         const uint32_t* kept_bits, void* out, cudaStream_t st) {
+    if (p.G * p.B >= 256 && !getenv("FP2_SINGLE_TILE"))
+        return launch_attn_pair(p, q, k, v, kept_bits, out, st);
     if (p.fp8) {
         if (p.d == 128 && p.B == 128) return launch_attn_t<128, 128, true>(p, q, k, v, kept_bits, out, st);
         return cudaErrorInvalidValue;

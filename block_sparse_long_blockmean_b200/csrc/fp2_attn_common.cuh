@@ -1,0 +1,168 @@
+// fp2_attn_common.cuh -- pieces shared by the two attention kernels:
+// tensor maps, the per-CTA work list (union of the G heads' kept blocks,
+// then the block-mean tiles that carry the correction), and the TMA issue of
+// one K/V (or mean) tile into a pipeline stage.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "fp2_seq.cuh"
+
+namespace fp2 {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
+constexpr float kRescaleLog2 = 8.0f;              // lazy-rescale threshold (x256)
+
+struct AttnMaps {
+    CUtensorMap q, k, v, kb, vb;
+};
+
+// Host: encodes the five tensor maps of an attention launch (Q boxes of
+// tok x G rows; K/V boxes of one key block or one page; mean-tile boxes).
+bool make_attn_maps(const KParams& p, const void* q, const void* k, const void* v, int D,
+                    int BLK, int TOK, AttnMaps* maps);
+
+// Loads the G heads' kept bits of query block i into sbits[G][nw_c] (block 0
+// and the diagonal forced on, bits past the diagonal cleared).  All threads.
+__device__ __forceinline__ void load_kept_bits(const KParams& p, const uint32_t* kept_bits, int b,
+                                               int hk, int i, int iabs, int nw_c, uint32_t* sbits) {
+    const int G = p.G;
+    const uint32_t* src = kept_bits + (((size_t)b * p.Hq + (size_t)hk * G) * p.nqb_max + i) * p.nw;
+    for (int x = threadIdx.x; x < G * nw_c; x += blockDim.x) {
+        const int g = x / nw_c, w = x % nw_c;
+        uint32_t word = src[(size_t)g * p.nqb_max * p.nw + w];
+        if (w == 0) word |= 1u;
+        if (w == (iabs >> 5)) {
+            word |= 1u << (iabs & 31);
+            const int hi = iabs & 31;
+            if (hi < 31) word &= (2u << hi) - 1u;
+        }
+        sbits[x] = word;
+    }
+}
+
+// One warp: writes the work list into items[] and returns its length.
+//   item >= 0 : key block j kept by at least one of the G heads (ascending)
+//   item <  0 : -(t+1), the tile of block means [t*BLK, t*BLK+BLK) that holds
+//               at least one block some head dropped (blocks < iabs)
+template <int BLK>
+__device__ __forceinline__ int build_items(int G, int iabs, int nw_c, const uint32_t* sbits,
+                                           int* items) {
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+    for (int w0 = 0; w0 < nw_c; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t u = 0;
+        if (w < nw_c)
+            for (int g = 0; g < G; ++g) u |= sbits[g * nw_c + w];
+        const int c = __popc(u);
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        int pos = base + incl - c;
+        while (u) {
+            const int bit = __ffs(u) - 1;
+            u &= u - 1;
+            items[pos++] = w * 32 + bit;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const int nvt = (iabs + BLK - 1) / BLK;
+    for (int t = 0; t < nvt; ++t) {
+        const int lo = t * BLK, hi = min(iabs, (t + 1) * BLK);  // blocks [lo, hi)
+        const int w_lo = lo >> 5, nwt = ((hi + 31) >> 5) - w_lo;
+        bool any = false;
+        for (int x = lane; x < G * nwt; x += 32) {
+            const int g = x / nwt, w = w_lo + x % nwt;
+            uint32_t m = ~sbits[g * nw_c + w];
+            const int top = hi - w * 32;  // > 0
+            if (top < 32) m &= (1u << top) - 1u;
+            any |= (m != 0u);
+        }
+        any = __any_sync(0xffffffffu, any);
+        if (lane == 0 && any) items[base] = -(t + 1);
+        if (any) ++base;
+    }
+    return base;
+}
+
+// Issues the TMA loads of one work item into a stage (K tile at k_s, V tile
+// at v_s; NCH 128-byte chunks of BLK rows each) and arms `full` with the
+// bytes that will land.  Paged keys load one box per page that holds keys of
+// the block; pages past the sequence end are skipped (their rows are never
+// used: the diagonal mask drops them and the V rows are zeroed).
+template <int D, int BLK, bool FP8>
+__device__ __forceinline__ void issue_item_loads(const KParams& p, const AttnMaps& maps,
+                                                 const SeqInfo& s, int b, int hk, int item,
+                                                 uint32_t k_s, uint32_t v_s, uint64_t* full) {
+    constexpr int ELT = FP8 ? 1 : 2;
+    constexpr int CH = 128 / ELT;
+    constexpr int NCH = D / CH;
+    constexpr int KV_BYTES = BLK * D * ELT;
+    if (item >= 0) {
+        const int j = item;
+        if (!p.paged) {
+            mbar_arrive_expect_tx(full, 2 * KV_BYTES);
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                tma_load_3d(k_s + c * BLK * 128, &maps.k, full, c * CH, hk, s.k0 + j * BLK);
+                tma_load_3d(v_s + c * BLK * 128, &maps.v, full, c * CH, hk, s.k0 + j * BLK);
+            }
+        } else {
+            const int R = min(p.page_size, BLK);
+            int nbox = 0;
+            int pages[BLK / 16];
+            for (int sb = 0; sb < BLK / R; ++sb) {
+                const int tok = j * BLK + sb * R;
+                int pg = -1;
+                if (tok < s.Lk) {
+                    pg = p.page_table[(size_t)b * p.max_pages + tok / p.page_size];
+                    if (pg < 0 || pg >= p.num_pages) {
+                        set_error(p.err, kErrBounds, kDetPage);
+                        pg = -1;
+                    }
+                }
+                pages[sb] = pg;
+                nbox += (pg >= 0);
+            }
+            mbar_arrive_expect_tx(full, (uint32_t)(2 * nbox * NCH * R * 128));
+            for (int sb = 0; sb < BLK / R; ++sb) {
+                if (pages[sb] < 0) continue;
+                const int off = (j * BLK + sb * R) % p.page_size;
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+                    tma_load_4d(k_s + c * BLK * 128 + sb * R * 128, &maps.k, full, c * CH, hk, off,
+                                pages[sb]);
+                    tma_load_4d(v_s + c * BLK * 128 + sb * R * 128, &maps.v, full, c * CH, hk, off,
+                                pages[sb]);
+                }
+            }
+        }
+    } else {
+        const int t = -item - 1;
+        mbar_arrive_expect_tx(full, 2 * KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            tma_load_3d(k_s + c * BLK * 128, &maps.kb, full, c * CH, t * BLK, b * p.Hkv + hk);
+            tma_load_3d(v_s + c * BLK * 128, &maps.vb, full, c * CH, t * BLK, b * p.Hkv + hk);
+        }
+    }
+}
+
+// Zeroes rows [nvalid, BLK) of a V tile (NCH chunks of BLK x 128 bytes) with
+// `nthr` cooperating threads (index `tid`).  Whole 128-byte rows are zeroed,
+// so the swizzle inside a row does not matter.
+template <int BLK, int NCH>
+__device__ __forceinline__ void zero_v_tail(uint8_t* v_tile, int nvalid, int tid, int nthr) {
+    const int units = (BLK - nvalid) * 8;  // 16-byte units per chunk
+    for (int c = 0; c < NCH; ++c)
+        for (int x16 = tid; x16 < units; x16 += nthr)
+            *reinterpret_cast<uint4*>(v_tile + c * BLK * 128 + nvalid * 128 + x16 * 16) =
+                make_uint4(0, 0, 0, 0);
+}
+
+}  // namespace fp2

@@ -1,0 +1,421 @@
+// fp2_attn_pair.cu -- the block-sparse attention kernel for query blocks of
+// at least 256 packed rows (G * block >= 256): two 128-row tiles per CTA
+// share every K/V tile and alternate on the tensor core.
+//
+// Same result as the single-tile kernel (fp2_attn.cu): for each query row an
+// online softmax over the tokens of the kept key blocks plus one pseudo-token
+// per dropped block (logit q.kbar/sqrt(d) + ln n_j, value vbar) -- the
+// FlashPrefill V2 abstract's sparse operator with PackGQA access and the
+// mean correction term.
+//
+// Work item = (sequence, KV head, query block i, pair index): tile A holds
+// tokens [t0, t0+TOK) x G heads, tile B the next TOK tokens (TOK = 128/G).
+// Both tiles belong to query block i, so they walk the same list of kept
+// blocks and mean tiles, and each K/V tile is loaded once for 256 rows.
+//
+// Roles (384 threads = 3 warpgroups; registers rebalanced with setmaxnreg:
+// 224 per softmax thread, 56 in the control warpgroup, 384 x 168 in total):
+//   warps 0-3  softmax for tile A (thread = row = TMEM lane)
+//   warps 4-7  softmax for tile B
+//   warp 8     TMA producer (both Q tiles, then the K/V ring of 2 stages)
+//   warps 10-11 idle
+//   warp 9     TMEM owner; lane 0 issues the MMAs in the order
+//                PV_A(n-1), QK_A(n), PV_B(n-1), QK_B(n)
+//              so that while one warpgroup works on its S the tensor core
+//              runs the other tile's two products.
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384),
+// O_B [384,512).  P_X (bf16 pairs or e4m3 quads) is written over the first
+// columns of S_X once the softmax has read S_X, and PV_X reads it from TMEM
+// (A operand in tensor memory).  QK_X(n+1) is issued after PV_X(n) by the
+// same thread; tcgen05.mma operations of one thread execute in issue order,
+// so PV_X(n) has read P_X before QK_X(n+1) overwrites it.  The commit that
+// signals S_X(n) full also covers PV_X(n-1), so when a softmax thread reads
+// S_X(n), O_X is stable and may be rescaled in place.
+#include "fp2_attn_common.cuh"
+
+namespace fp2 {
+
+template <int D, int BLK, bool FP8>
+struct PairCfg {
+    static constexpr int ELT = FP8 ? 1 : 2;
+    static constexpr int CH = 128 / ELT;
+    static constexpr int NCH = D / CH;
+    static constexpr int KSTEP = FP8 ? 32 : 16;
+    static constexpr int Q_BYTES = 128 * D * ELT;   // one tile
+    static constexpr int KV_BYTES = BLK * D * ELT;
+    static constexpr int P_COLS = BLK * ELT / 4;    // 32-bit TMEM columns of one P row
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = 2 * Q_BYTES;
+    static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
+    static constexpr int OFF_MISC = OFF_BAR + 256;
+    static constexpr int OFF_ITEMS = OFF_MISC + 64;
+    static_assert(P_COLS % 32 == 0, "P row must be whole 32-column TMEM stores");
+};
+
+enum { PB_KV_FULL = 0, PB_KV_EMPTY = 2, PB_Q_FULL = 4, PB_S_FULL = 5, PB_P_READY = 7,
+       PB_O_FINAL = 9, PB_DRAIN = 11, PB_COUNT = 12 };
+
+template <int D, int BLK, bool FP8>
+__global__ void __launch_bounds__(384, 1)
+attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
+                 const uint32_t* __restrict__ kept_bits, __nv_bfloat16* __restrict__ out,
+                 int items_cap) {
+    using C = PairCfg<D, BLK, FP8>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+    int* items = reinterpret_cast<int*>(smem + C::OFF_ITEMS);
+    uint32_t* sbits = reinterpret_cast<uint32_t*>(items + items_cap);
+
+    const int G = p.G;
+    const int TOK = 128 / G;
+    const int npair = BLK / (2 * TOK);
+    const int per_i = p.num_seqs * p.Hkv * npair;
+    const int i = p.nqb_max - 1 - (int)(blockIdx.x / per_i);  // longest first
+    const int rem = (int)(blockIdx.x % per_i);
+    const int b = rem / (p.Hkv * npair);
+    const int hk = (rem / npair) % p.Hkv;
+    const int pr = rem % npair;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    SeqInfo s;
+    if (!load_seq(p, b, s)) return;
+    const int t_begin = i * BLK + pr * 2 * TOK;
+    if (t_begin >= s.Lq) return;
+    const int iabs = s.P / BLK + i;
+    const int nw_c = (iabs + 32) / 32;
+
+    if (threadIdx.x == 0) {
+        for (int k = 0; k < PB_COUNT; ++k)
+            mbar_init(&bars[k], (k == PB_P_READY || k == PB_P_READY + 1) ? 128u : 1u);
+        misc[1] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(&misc[0], 512);
+        tmem_relinquish();
+    }
+    load_kept_bits(p, kept_bits, b, hk, i, iabs, nw_c, sbits);
+    __syncthreads();
+    if (warp == 8) {
+        const int n = build_items<BLK>(G, iabs, nw_c, sbits, items);
+        if (lane == 0) misc[2] = (uint32_t)n;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    const int n_items = (int)misc[2];
+    const uint32_t q_s = sbase + C::OFF_Q;
+
+    if (warp >= 8) {
+      regs_decrease<56>();
+      if (warp == 8 && lane == 0) {
+        // ---------------------------------------------------------- producer ---
+            prefetch_tmap(&maps.q);
+            prefetch_tmap(&maps.k);
+            prefetch_tmap(&maps.v);
+            mbar_arrive_expect_tx(&bars[PB_Q_FULL], 2 * C::Q_BYTES);
+            for (int x = 0; x < 2; ++x)
+                for (int c = 0; c < C::NCH; ++c)
+                    tma_load_3d(q_s + x * C::Q_BYTES + c * (128 * 128), &maps.q, &bars[PB_Q_FULL],
+                                c * C::CH, hk * G, s.q0 + t_begin + x * TOK);
+            int issued = 0;
+            for (int n = 0; n < n_items; ++n) {
+                const int st = n & 1;
+                if (n >= 2 && !mbar_wait(&bars[PB_KV_EMPTY + st], ((n - 2) >> 1) & 1, abort_flag,
+                                         kWaitLimitNs)) {
+                    set_error(p.err, kErrTimeout, kDetWaitBase + 0);
+                    break;
+                }
+                issue_item_loads<D, BLK, FP8>(p, maps, s, b, hk, items[n],
+                                              sbase + C::OFF_K + st * C::KV_BYTES,
+                                              sbase + C::OFF_V + st * C::KV_BYTES,
+                                              &bars[PB_KV_FULL + st]);
+                ++issued;
+            }
+            volatile int no_abort = 0;
+            for (int n = max(0, issued - 2); n < issued; ++n)
+                mbar_wait(&bars[PB_KV_FULL + (n & 1)], (n >> 1) & 1, &no_abort, kWaitLimitNs);
+            mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, kWaitLimitNs);
+      } else if (warp == 9 && lane == 0) {
+        // -------------------------------------------------------------- MMA ---
+            constexpr uint32_t fmt = FP8 ? 0u : 1u;
+            constexpr uint32_t idesc_qk = make_idesc(fmt, false, 128, BLK);
+            constexpr uint32_t idesc_pv = make_idesc(fmt, true, 128, D);
+            bool ok = mbar_wait(&bars[PB_Q_FULL], 0, abort_flag, kWaitLimitNs);
+            if (!ok) set_error(p.err, kErrTimeout, kDetWaitBase + 1);
+            tc_fence_after();
+            for (int n = 0; ok && n <= n_items; ++n) {
+                const int st = n & 1;
+                if (n < n_items &&
+                    !mbar_wait(&bars[PB_KV_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs)) {
+                    set_error(p.err, kErrTimeout, kDetWaitBase + 2);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int x = 0; x < 2; ++x) {
+                    if (n >= 1) {
+                        const int m = n - 1;
+                        if (!mbar_wait(&bars[PB_P_READY + x], m & 1, abort_flag, kWaitLimitNs)) {
+                            set_error(p.err, kErrTimeout, kDetWaitBase + 3);
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t v_s = sbase + C::OFF_V + (m & 1) * C::KV_BYTES;
+                        const uint32_t p_tmem = tmem + x * 128;
+                        const uint32_t o_tmem = tmem + 256 + x * 128;
+#pragma unroll
+                        for (int ks = 0; ks < BLK / C::KSTEP; ++ks) {
+                            const uint64_t bd =
+                                sw128_desc(v_s + ks * C::KSTEP * 128, BLK * 128, 1024);
+                            const uint32_t acc = (m > 0 || ks > 0) ? 1u : 0u;
+                            if constexpr (FP8) mma_f8_ts(o_tmem, p_tmem + ks * 8, bd, idesc_pv, acc);
+                            else mma_bf16_ts(o_tmem, p_tmem + ks * 8, bd, idesc_pv, acc);
+                        }
+                        if (x == 1) mma_commit(&bars[PB_KV_EMPTY + (m & 1)]);
+                        if (m == n_items - 1) mma_commit(&bars[PB_O_FINAL + x]);
+                    }
+                    if (n < n_items) {
+                        const uint32_t k_s = sbase + C::OFF_K + st * C::KV_BYTES;
+                        const uint32_t qx = q_s + x * C::Q_BYTES;
+                        const uint32_t s_tmem = tmem + x * 128;
+#pragma unroll
+                        for (int ks = 0; ks < D / C::KSTEP; ++ks) {
+                            const int ch = (ks * C::KSTEP) / C::CH;
+                            const uint32_t within = (uint32_t)((ks * C::KSTEP) % C::CH) * C::ELT;
+                            const uint64_t ad = sw128_desc(qx + ch * (128 * 128) + within, 16, 1024);
+                            const uint64_t bd =
+                                sw128_desc(k_s + ch * (BLK * 128) + within, 16, 1024);
+                            if constexpr (FP8) mma_f8_ss(s_tmem, ad, bd, idesc_qk, ks > 0);
+                            else mma_bf16_ss(s_tmem, ad, bd, idesc_qk, ks > 0);
+                        }
+                        mma_commit(&bars[PB_S_FULL + x]);
+                    }
+                }
+            }
+            mma_commit(&bars[PB_DRAIN]);
+            volatile int no_abort = 0;
+            mbar_wait(&bars[PB_DRAIN], 0, &no_abort, kWaitLimitNs);
+      }
+    } else {
+        regs_increase<224>();
+        // ---------------------------------------------------------- softmax ---
+        const int X = warp >> 2;                  // tile
+        const int qw = warp & 3;
+        const int r = qw * 32 + lane;             // row of the tile == TMEM lane
+        const int g = r % G;
+        const int t = t_begin + X * TOK + r / G;  // query index in the sequence
+        const int h = hk * G + g;
+        const bool row_ok = t < s.Lq;
+        const int ppos = s.P + t;
+        const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + X * 128;
+        const uint32_t o_addr = tmem + lane_off + 256 + X * 128;
+        const uint32_t* hb = sbits + g * nw_c;
+        float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
+        if constexpr (FP8) sl2 *= p.q_scale[h] * p.k_scale[hk];
+        const float lb = __log2f((float)BLK);
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int n = 0; n < n_items; ++n) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[PB_S_FULL + X], n & 1, abort_flag,
+                                                   kWaitLimitNs))) {
+                set_error(p.err, kErrTimeout, kDetWaitBase + 4);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float x[BLK];
+#pragma unroll
+            for (int c = 0; c < BLK / 32; ++c) tmem_ld32f(s_addr + c * 32, x + c * 32);
+            tmem_wait_ld();
+
+            const int item = items[n];
+            float mx = -INFINITY;
+            if (item >= 0) {
+                const int j = item;
+                const bool kept = row_ok && ((hb[j >> 5] >> (j & 31)) & 1u);
+                const int lim = !kept ? -1 : (j == iabs ? ppos - j * BLK : BLK - 1);
+                if (lim == BLK - 1) {
+#pragma unroll
+                    for (int c = 0; c < BLK; ++c) {
+                        x[c] *= sl2;
+                        mx = fmaxf(mx, x[c]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BLK; ++c) {
+                        const float v = c <= lim ? x[c] * sl2 : -INFINITY;
+                        x[c] = v;
+                        mx = fmaxf(mx, v);
+                    }
+                }
+            } else {
+                const int tv = -item - 1;
+#pragma unroll
+                for (int c0 = 0; c0 < BLK; c0 += 32) {
+                    const int j0 = tv * BLK + c0;
+                    uint32_t dropped = 0u;
+                    if (row_ok && j0 < iabs) {
+                        dropped = ~hb[j0 >> 5];
+                        const int nvalid = iabs - j0;
+                        if (nvalid < 32) dropped &= (1u << nvalid) - 1u;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float v = ((dropped >> e) & 1u) ? fmaf(x[c0 + e], sl2, lb) : -INFINITY;
+                        x[c0 + e] = v;
+                        mx = fmaxf(mx, v);
+                    }
+                }
+            }
+            float alpha = 1.f;
+            bool rescale = false;
+            if (m_used == -INFINITY) {
+                m_used = mx;
+            } else if (mx > m_used + kRescaleLog2) {
+                alpha = ex2(m_used - mx);
+                m_used = mx;
+                rescale = true;
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O_X is stable here (PV_X(n-1) completed before S_X(n) was signalled)
+                const float a = rescale ? alpha : 1.f;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + c * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
+                    tmem_st32(o_addr + c * 32, o);
+                }
+            }
+            const float mb = m_used == -INFINITY ? 0.f : m_used;
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+            for (int c = 0; c < BLK; c += 4) {
+                x[c] = ex2(x[c] - mb);
+                x[c + 1] = ex2(x[c + 1] - mb);
+                x[c + 2] = ex2(x[c + 2] - mb);
+                x[c + 3] = ex2(x[c + 3] - mb);
+                s0 += x[c];
+                s1 += x[c + 1];
+                s2 += x[c + 2];
+                s3 += x[c + 3];
+            }
+            l = l * alpha + ((s0 + s1) + (s2 + s3));
+            // P_X -> TMEM over S_X
+#pragma unroll
+            for (int c = 0; c < C::P_COLS / 32; ++c) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    if constexpr (FP8) {
+                        const float* src = x + (c * 32 + e) * 4;
+                        const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+                            make_float2(src[0], src[1]), __NV_SATFINITE, __NV_E4M3);
+                        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+                            make_float2(src[2], src[3]), __NV_SATFINITE, __NV_E4M3);
+                        pk[e] = (uint32_t)lo | ((uint32_t)hi << 16);
+                    } else {
+                        __nv_bfloat162 hh = __floats2bfloat162_rn(x[(c * 32 + e) * 2],
+                                                                  x[(c * 32 + e) * 2 + 1]);
+                        pk[e] = *reinterpret_cast<uint32_t*>(&hh);
+                    }
+                }
+                tmem_st32(s_addr + c * 32, pk);
+            }
+            if (X == 0 && item >= 0 && item * BLK + BLK > s.Lk) {
+                zero_v_tail<BLK, C::NCH>(smem + C::OFF_V + (n & 1) * C::KV_BYTES,
+                                         max(0, s.Lk - item * BLK), r, 128);
+                fence_proxy_async_smem();
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[PB_P_READY + X]);
+        }
+        if (ok && __all_sync(0xffffffffu, mbar_wait(&bars[PB_O_FINAL + X], 0, abort_flag,
+                                                    kWaitLimitNs))) {
+            tc_fence_after();
+            float inv = l > 0.f ? 1.f / l : 0.f;
+            if constexpr (FP8) inv *= p.v_scale[hk];
+            __nv_bfloat16* orow = out + ((size_t)(s.q0 + t) * p.Hq + h) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(o_addr + c * 32, o);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        uint32_t wd[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            __nv_bfloat162 hh = __floats2bfloat162_rn(
+                                __uint_as_float(o[u * 8 + 2 * e]) * inv,
+                                __uint_as_float(o[u * 8 + 2 * e + 1]) * inv);
+                            wd[e] = *reinterpret_cast<uint32_t*>(&hh);
+                        }
+                        *reinterpret_cast<uint4*>(orow + c * 32 + u * 8) =
+                            make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                    }
+                }
+            }
+        } else if (ok) {
+            set_error(p.err, kErrTimeout, kDetWaitBase + 6);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D, int BLK, bool FP8>
+cudaError_t launch_attn_pair_t(const KParams& p, const void* q, const void* k, const void* v,
+                               const uint32_t* kept_bits, void* out, cudaStream_t st) {
+    using C = PairCfg<D, BLK, FP8>;
+    AttnMaps maps;
+    const int TOK = 128 / p.G;
+    if (!make_attn_maps(p, q, k, v, D, BLK, TOK, &maps)) return cudaErrorInvalidValue;
+    const int items_cap = p.nkb_max + (p.nkb_max + BLK - 1) / BLK + 2;
+    const int nw_c_max = p.nkb_max / 32 + 1;
+    size_t smem = 1024 + C::OFF_ITEMS + (size_t)items_cap * 4 + (size_t)p.G * nw_c_max * 4;
+    if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM: it owns all 512 TMEM columns
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(attn_pair_kernel<D, BLK, FP8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int npair = BLK / (2 * TOK);
+    const long long grid = (long long)p.nqb_max * p.num_seqs * p.Hkv * npair;
+    if (grid <= 0) return cudaSuccess;
+    attn_pair_kernel<D, BLK, FP8><<<(unsigned)grid, 384, smem, st>>>(
+        p, maps, kept_bits, static_cast<__nv_bfloat16*>(out), items_cap);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_pair(const KParams& p, const void* q, const void* k, const void* v,
+                             const uint32_t* kept_bits, void* out, cudaStream_t st) {
+    if (p.fp8) {
+        if (p.d == 128 && p.B == 128) return launch_attn_pair_t<128, 128, true>(p, q, k, v, kept_bits, out, st);
+        return cudaErrorInvalidValue;
+    }
+    if (p.d == 128 && p.B == 128) return launch_attn_pair_t<128, 128, false>(p, q, k, v, kept_bits, out, st);
+    if (p.d == 128 && p.B == 64) return launch_attn_pair_t<128, 64, false>(p, q, k, v, kept_bits, out, st);
+    if (p.d == 64 && p.B == 128) return launch_attn_pair_t<64, 128, false>(p, q, k, v, kept_bits, out, st);
+    if (p.d == 64 && p.B == 64) return launch_attn_pair_t<64, 64, false>(p, q, k, v, kept_bits, out, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace fp2
