@@ -137,6 +137,18 @@ def algorithmic_flops(cnt, lens_q, lens_k, B, d):
     return kept_fl, corr_fl, dropped / max(causal, 1)
 
 
+def union_inflation(words, cnt, Hkv):
+    """PackGQA walks the union of the G heads' kept blocks: (union size x G)
+    summed over (sequence, KV head, query block) / kept blocks summed over
+    heads.  1.0 = every head of a group keeps the same blocks."""
+    S, Hq, nqb, nw = words.shape
+    G = Hq // Hkv
+    u = np.bitwise_or.reduce(words.reshape(S, Hkv, G, nqb, nw), axis=2)
+    pop = np.unpackbits(u.view(np.uint8), axis=-1).sum(axis=(-1, -2), dtype=np.int64)
+    kept = int(cnt.astype(np.int64).sum())
+    return float(pop.sum() * G) / max(kept, 1)
+
+
 def dense_flops(lens_q, lens_k, Hq, d):
     """Exact-causal dense flops: 4*d per (query, visible key) pair."""
     f = 0.0
@@ -202,6 +214,8 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
         L = pr.layout()
         cnt = pr.ws_view("kept_cnt", torch.int32, (inp.num_seqs, s.Hq, L.nqb_max)).cpu().numpy()
         kept_fl, corr_fl, drop_frac = algorithmic_flops(cnt, s.lens_q, s.lens_k, B, s.d)
+        words = pr.ws_view("kept_bits", torch.int32, (inp.num_seqs, s.Hq, L.nqb_max, L.nw))
+        union_ratio = union_inflation(words.cpu().numpy().view(np.uint32), cnt, s.Hkv)
 
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
         if world > 1:
@@ -271,6 +285,7 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
         "stage_ms": {"blockmean": stage_ms[0], "score": stage_ms[1], "mask": stage_ms[2],
                      "attn": stage_ms[3]},
         "kept_flops": kept_fl, "corr_flops": corr_fl, "clocks": clk, "dense": dense,
+        "union_inflation": union_ratio,
         "e2e": e2e, "gen_s": gen_s, "inp": inp if want_cpu else None, "tau_inp": tau,
     }
     return res
@@ -404,6 +419,8 @@ def main():
                "tensor_peak_frac_measured": eff / peak,
                "tensor_peak_frac_datasheet": eff / (2250.0 * (2.0 if x["dtype"] == "fp8" else 1.0)),
                "drop_fraction": x["drop_fraction"], "tau": x["tau"],
+               "union_inflation": x["union_inflation"],
+               "tensor_frac_executed_measured": eff * x["union_inflation"] / peak,
                "stage_ms": x["stage_ms"],
                "prefill_roofline_frac": (x["kept_flops"] / peak / 1e12) / (x["ms_per_step"] * 1e-3)}
         if x["dense"]:

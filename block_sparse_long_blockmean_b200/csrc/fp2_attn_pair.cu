@@ -233,33 +233,30 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 break;
             }
             tc_fence_after();
-            float x[BLK];
+            float2 xv[BLK / 2];  // the row's scores as aligned pairs
+            float* x = reinterpret_cast<float*>(xv);
 #pragma unroll
             for (int c = 0; c < BLK / 32; ++c) tmem_ld32f(s_addr + c * 32, x + c * 32);
             tmem_wait_ld();
 
             const int item = items[n];
-            float mx = -INFINITY;
+            // Masks act on raw scores (the scale sl2 is positive); the bias
+            // of a mean tile (log2 n_j) and the running max fold into the one
+            // FFMA that feeds exp2:  p = 2^(x * sl2 + (bias - m)).
+            bool live;       // this row takes part in this item
+            float bias = 0.f;
             if (item >= 0) {
                 const int j = item;
-                const bool kept = row_ok && ((hb[j >> 5] >> (j & 31)) & 1u);
-                const int lim = !kept ? -1 : (j == iabs ? ppos - j * BLK : BLK - 1);
-                if (lim == BLK - 1) {
+                live = row_ok && ((hb[j >> 5] >> (j & 31)) & 1u);
+                if (live && j == iabs) {
+                    const int lim = ppos - j * BLK;
 #pragma unroll
-                    for (int c = 0; c < BLK; ++c) {
-                        x[c] *= sl2;
-                        mx = fmaxf(mx, x[c]);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < BLK; ++c) {
-                        const float v = c <= lim ? x[c] * sl2 : -INFINITY;
-                        x[c] = v;
-                        mx = fmaxf(mx, v);
-                    }
+                    for (int c = 0; c < BLK; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
                 }
             } else {
                 const int tv = -item - 1;
+                bias = lb;
+                live = false;
 #pragma unroll
                 for (int c0 = 0; c0 < BLK; c0 += 32) {
                     const int j0 = tv * BLK + c0;
@@ -269,13 +266,25 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                         const int nvalid = iabs - j0;
                         if (nvalid < 32) dropped &= (1u << nvalid) - 1u;
                     }
+                    live |= dropped != 0u;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float v = ((dropped >> e) & 1u) ? fmaf(x[c0 + e], sl2, lb) : -INFINITY;
-                        x[c0 + e] = v;
-                        mx = fmaxf(mx, v);
-                    }
+                    for (int e = 0; e < 32; ++e)
+                        x[c0 + e] = ((dropped >> e) & 1u) ? x[c0 + e] : -INFINITY;
                 }
+            }
+            float mx = -INFINITY;
+            if (live) {
+                float m0 = x[0], m1 = x[1], m2 = x[2], m3 = x[3];
+#pragma unroll
+                for (int c = 4; c < BLK; c += 8) {
+                    m0 = max3f(m0, x[c], x[c + 1]);
+                    m1 = max3f(m1, x[c + 2], x[c + 3]);
+                    m2 = max3f(m2, x[c + 4], x[c + 5]);
+                    if (c + 7 < BLK) m3 = max3f(m3, x[c + 6], x[c + 7]);
+                    else m3 = fmaxf(m3, x[c + 6]);
+                }
+                mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+                if (mx != -INFINITY) mx = fmaf(mx, sl2, bias);
             }
             float alpha = 1.f;
             bool rescale = false;
@@ -299,20 +308,24 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                     tmem_st32(o_addr + c * 32, o);
                 }
             }
-            const float mb = m_used == -INFINITY ? 0.f : m_used;
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            float sum = 0.f;
+            {
+                // a row that takes no part gets offset -inf: every p is 0
+                const float c0 = live ? bias - m_used : -INFINITY;
+                const float2 k2 = make_float2(sl2, sl2), c2 = make_float2(c0, c0);
+                float2 a0 = make_float2(0.f, 0.f), a1 = a0;
 #pragma unroll
-            for (int c = 0; c < BLK; c += 4) {
-                x[c] = ex2(x[c] - mb);
-                x[c + 1] = ex2(x[c + 1] - mb);
-                x[c + 2] = ex2(x[c + 2] - mb);
-                x[c + 3] = ex2(x[c + 3] - mb);
-                s0 += x[c];
-                s1 += x[c + 1];
-                s2 += x[c + 2];
-                s3 += x[c + 3];
+                for (int c = 0; c < BLK / 2; c += 2) {
+                    float2 e0 = ffma2(xv[c], k2, c2);
+                    float2 e1 = ffma2(xv[c + 1], k2, c2);
+                    xv[c] = make_float2(ex2(e0.x), ex2(e0.y));
+                    xv[c + 1] = make_float2(ex2(e1.x), ex2(e1.y));
+                    a0 = fadd2(a0, xv[c]);
+                    a1 = fadd2(a1, xv[c + 1]);
+                }
+                sum = (a0.x + a0.y) + (a1.x + a1.y);
             }
-            l = l * alpha + ((s0 + s1) + (s2 + s3));
+            l = l * alpha + sum;
             // P_X -> TMEM over S_X
 #pragma unroll
             for (int c = 0; c < C::P_COLS / 32; ++c) {
@@ -321,15 +334,9 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 for (int e = 0; e < 32; ++e) {
                     if constexpr (FP8) {
                         const float* src = x + (c * 32 + e) * 4;
-                        const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-                            make_float2(src[0], src[1]), __NV_SATFINITE, __NV_E4M3);
-                        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-                            make_float2(src[2], src[3]), __NV_SATFINITE, __NV_E4M3);
-                        pk[e] = (uint32_t)lo | ((uint32_t)hi << 16);
+                        pk[e] = pack_e4m3x4(src[0], src[1], src[2], src[3]);
                     } else {
-                        __nv_bfloat162 hh = __floats2bfloat162_rn(x[(c * 32 + e) * 2],
-                                                                  x[(c * 32 + e) * 2 + 1]);
-                        pk[e] = *reinterpret_cast<uint32_t*>(&hh);
+                        pk[e] = pack_bf16x2(x[(c * 32 + e) * 2], x[(c * 32 + e) * 2 + 1]);
                     }
                 }
                 tmem_st32(s_addr + c * 32, pk);

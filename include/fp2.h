@@ -42,6 +42,10 @@
  *    G = Hq/Hkv in {1,2,4,8} with 128/G <= block, page_size a power of two
  *    in [16, 256] that divides the block or is divided by it.
  *
+ * Kernel choice: problems with G * block >= 256 packed rows per query block
+ * run the two-tile attention kernel, smaller ones the one-tile kernel; the
+ * environment variable FP2_SINGLE_TILE=1 forces the one-tile kernel (tests).
+ *
  * Errors: argument errors are returned synchronously before any launch.
  * CUDA launch errors return FP2_ERR_CUDA.  Problems only the device can see
  * (a prefix that is not a multiple of the block, Lk < Lq, a length above

@@ -247,3 +247,22 @@ def test_calibrate_tau_matches_target():
                 for r in orc)
     kept = int(got.sum())
     assert abs((total - kept) - round(0.7 * total)) <= 2
+
+
+@pytest.mark.parametrize("name", ["tiny_1k_d64_b64", "varlen_paged64_fp8", "chunk_prefix_g8",
+                                  "ragged_2k_g4"])
+def test_single_tile_kernel_on_large_groups(name, monkeypatch):
+    """FP2_SINGLE_TILE=1 routes G*block >= 256 problems to the one-tile kernel
+    too, so both attention kernels are checked on the same cases."""
+    monkeypatch.setenv("FP2_SINGLE_TILE", "1")
+    inp = make_inputs(name)
+    orc = H.oracle_scores(inp)
+    tau = H.pick_tau(orc, inp.shape.drop)
+    pr = H.problem(inp, out_fill=float("nan"))
+    pr.prefill(tau)
+    pr.check()
+    for b in range(inp.num_seqs):
+        keep = O.mask(orc[b][3], orc[b][4], tau)
+        ref, _, _ = H.oracle_out(inp, b, orc[b], keep)
+        H.assert_close(H.out_seq(pr, inp, b).reshape(ref.shape), ref, inp.shape.dtype == "fp8",
+                       f"{name} seq {b}")
