@@ -51,6 +51,15 @@ struct PairCfg {
     static constexpr int OFF_MISC = OFF_BAR + 256;
     static constexpr int OFF_ITEMS = OFF_MISC + 64;
     static_assert(P_COLS % 32 == 0, "P row must be whole 32-column TMEM stores");
+    // pairs (of every 4) whose exp2 runs on the FMA pipe: the fp8 MMA is twice
+    // as fast, so more of the exp2 work moves off the MUFU unit there
+#ifndef FP2_EMU_PAIRS_FP8
+#define FP2_EMU_PAIRS_FP8 1
+#endif
+#ifndef FP2_EMU_PAIRS_BF16
+#define FP2_EMU_PAIRS_BF16 0
+#endif
+    static constexpr int kEmuPairs = FP8 ? FP2_EMU_PAIRS_FP8 : FP2_EMU_PAIRS_BF16;
 };
 
 enum { PB_KV_FULL = 0, PB_KV_EMPTY = 2, PB_Q_FULL = 4, PB_S_FULL = 5, PB_P_READY = 7,
@@ -314,14 +323,18 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 const float c0 = live ? bias - m_used : -INFINITY;
                 const float2 k2 = make_float2(sl2, sl2), c2 = make_float2(c0, c0);
                 float2 a0 = make_float2(0.f, 0.f), a1 = a0;
+                // of every 4 pairs, the last kEmuPairs go to the FMA pipe
+                // (exp2_poly2), the rest to MUFU ex2: the two units share the load
 #pragma unroll
-                for (int c = 0; c < BLK / 2; c += 2) {
-                    float2 e0 = ffma2(xv[c], k2, c2);
-                    float2 e1 = ffma2(xv[c + 1], k2, c2);
-                    xv[c] = make_float2(ex2(e0.x), ex2(e0.y));
-                    xv[c + 1] = make_float2(ex2(e1.x), ex2(e1.y));
-                    a0 = fadd2(a0, xv[c]);
-                    a1 = fadd2(a1, xv[c + 1]);
+                for (int c = 0; c < BLK / 2; c += 4) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 e = ffma2(xv[c + u], k2, c2);
+                        xv[c + u] = (u >= 4 - C::kEmuPairs) ? exp2_poly2(e)
+                                                             : make_float2(ex2(e.x), ex2(e.y));
+                        if (u & 1) a1 = fadd2(a1, xv[c + u]);
+                        else a0 = fadd2(a0, xv[c + u]);
+                    }
                 }
                 sum = (a0.x + a0.y) + (a1.x + a1.y);
             }

@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "fp2_exp2_poly.h"
+
 namespace fp2 {
 
 // ---------------------------------------------------------------- errors ---
@@ -295,6 +297,28 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(lo) : "f"(a), "f"(b));
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(hi) : "f"(c), "f"(d));
     return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// 2^x for a pair, on the FMA and integer pipes instead of the MUFU unit.
+// Cody-Waite reduction x = j + f (j = rint(x) by adding 1.5*2^23, exact for
+// |x| < 2^22), 2^f by the degree-3 polynomial of fp2_exp2_poly.h (relative
+// error < FP2_EXP2_REL_ERR on [-1/2, 1/2]), 2^j added to the exponent field.
+// Inputs are clamped to >= -126 so the exponent never wraps: anything below
+// (including -inf and NaN) returns a value <= 2^-125, i.e. a zero weight.
+// Valid for x <= 127.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    const float magic = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -126.0f);
+    x.y = fmaxf(x.y, -126.0f);
+    const float2 t = fadd2(x, make_float2(magic, magic));
+    const float2 j = fadd2(t, make_float2(-magic, -magic));
+    const float2 f = fadd2(x, make_float2(-j.x, -j.y));
+    float2 p = ffma2(f, make_float2(FP2_EXP2_C3, FP2_EXP2_C3),
+                     make_float2(FP2_EXP2_C2, FP2_EXP2_C2));
+    p = ffma2(p, f, make_float2(FP2_EXP2_C1, FP2_EXP2_C1));
+    p = ffma2(p, f, make_float2(FP2_EXP2_C0, FP2_EXP2_C0));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ float ex2(float x) {
