@@ -90,28 +90,31 @@ __device__ __forceinline__ int build_items(int G, int iabs, int nw_c, const uint
     return base;
 }
 
-// Issues the TMA loads of one work item into a stage (K tile at k_s, V tile
-// at v_s; NCH 128-byte chunks of BLK rows each) and arms `full` with the
-// bytes that will land.  Paged keys load one box per page that holds keys of
-// the block; pages past the sequence end are skipped (their rows are never
-// used: the diagonal mask drops them and the V rows are zeroed).
+// Issues the TMA loads of ONE operand tile of a work item (the K tile, or
+// the V tile: `map`/`mean_map` select which) into `dst` (NCH 128-byte chunks
+// of BLK rows) and adds the bytes that will land to `full`'s current phase.
+// `arrive`: also arrive on `full` (its arrival count is 1, so exactly one
+// call per phase may arrive; others only add their bytes).  Paged keys
+// load one box per page that holds keys of the block; pages past the
+// sequence end are skipped (their rows are never used: the diagonal mask
+// drops them and the V rows are zeroed).
 template <int D, int BLK, bool FP8>
-__device__ __forceinline__ void issue_item_loads(const KParams& p, const AttnMaps& maps,
-                                                 const SeqInfo& s, int b, int hk, int item,
-                                                 uint32_t k_s, uint32_t v_s, uint64_t* full) {
+__device__ __forceinline__ void issue_tile_load(const KParams& p, const CUtensorMap* map,
+                                                const CUtensorMap* mean_map, const SeqInfo& s,
+                                                int b, int hk, int item, uint32_t dst,
+                                                uint64_t* full, bool arrive) {
     constexpr int ELT = FP8 ? 1 : 2;
     constexpr int CH = 128 / ELT;
     constexpr int NCH = D / CH;
-    constexpr int KV_BYTES = BLK * D * ELT;
+    constexpr int TILE_BYTES = BLK * D * ELT;
     if (item >= 0) {
         const int j = item;
         if (!p.paged) {
-            mbar_arrive_expect_tx(full, 2 * KV_BYTES);
+            if (arrive) mbar_arrive_expect_tx(full, TILE_BYTES);
+            else mbar_expect_tx(full, TILE_BYTES);
 #pragma unroll
-            for (int c = 0; c < NCH; ++c) {
-                tma_load_3d(k_s + c * BLK * 128, &maps.k, full, c * CH, hk, s.k0 + j * BLK);
-                tma_load_3d(v_s + c * BLK * 128, &maps.v, full, c * CH, hk, s.k0 + j * BLK);
-            }
+            for (int c = 0; c < NCH; ++c)
+                tma_load_3d(dst + c * BLK * 128, map, full, c * CH, hk, s.k0 + j * BLK);
         } else {
             const int R = min(p.page_size, BLK);
             int nbox = 0;
@@ -129,28 +132,35 @@ __device__ __forceinline__ void issue_item_loads(const KParams& p, const AttnMap
                 pages[sb] = pg;
                 nbox += (pg >= 0);
             }
-            mbar_arrive_expect_tx(full, (uint32_t)(2 * nbox * NCH * R * 128));
+            if (arrive) mbar_arrive_expect_tx(full, (uint32_t)(nbox * NCH * R * 128));
+            else mbar_expect_tx(full, (uint32_t)(nbox * NCH * R * 128));
             for (int sb = 0; sb < BLK / R; ++sb) {
                 if (pages[sb] < 0) continue;
                 const int off = (j * BLK + sb * R) % p.page_size;
 #pragma unroll
-                for (int c = 0; c < NCH; ++c) {
-                    tma_load_4d(k_s + c * BLK * 128 + sb * R * 128, &maps.k, full, c * CH, hk, off,
+                for (int c = 0; c < NCH; ++c)
+                    tma_load_4d(dst + c * BLK * 128 + sb * R * 128, map, full, c * CH, hk, off,
                                 pages[sb]);
-                    tma_load_4d(v_s + c * BLK * 128 + sb * R * 128, &maps.v, full, c * CH, hk, off,
-                                pages[sb]);
-                }
             }
         }
     } else {
         const int t = -item - 1;
-        mbar_arrive_expect_tx(full, 2 * KV_BYTES);
+        if (arrive) mbar_arrive_expect_tx(full, TILE_BYTES);
+        else mbar_expect_tx(full, TILE_BYTES);
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-            tma_load_3d(k_s + c * BLK * 128, &maps.kb, full, c * CH, t * BLK, b * p.Hkv + hk);
-            tma_load_3d(v_s + c * BLK * 128, &maps.vb, full, c * CH, t * BLK, b * p.Hkv + hk);
-        }
+        for (int c = 0; c < NCH; ++c)
+            tma_load_3d(dst + c * BLK * 128, mean_map, full, c * CH, t * BLK, b * p.Hkv + hk);
     }
+}
+
+// Both tiles of a work item into one stage, one barrier: the K tile only
+// adds its bytes, the V tile adds its bytes and arrives (once per phase).
+template <int D, int BLK, bool FP8>
+__device__ __forceinline__ void issue_item_loads(const KParams& p, const AttnMaps& maps,
+                                                 const SeqInfo& s, int b, int hk, int item,
+                                                 uint32_t k_s, uint32_t v_s, uint64_t* full) {
+    issue_tile_load<D, BLK, FP8>(p, &maps.k, &maps.kb, s, b, hk, item, k_s, full, false);
+    issue_tile_load<D, BLK, FP8>(p, &maps.v, &maps.vb, s, b, hk, item, v_s, full, true);
 }
 
 // Zeroes rows [nvalid, BLK) of a V tile (NCH chunks of BLK x 128 bytes) with

@@ -62,8 +62,11 @@ struct PairCfg {
     static constexpr int kEmuPairs = FP8 ? FP2_EMU_PAIRS_FP8 : FP2_EMU_PAIRS_BF16;
 };
 
-enum { PB_KV_FULL = 0, PB_KV_EMPTY = 2, PB_Q_FULL = 4, PB_S_FULL = 5, PB_P_READY = 7,
-       PB_O_FINAL = 9, PB_DRAIN = 11, PB_COUNT = 12 };
+// K and V have separate rings: K(n) is free once QK_B(n) has run, V(n) only
+// after PV_B(n) -- a full MMA pair later -- so each stream refills as soon as
+// its own operand is consumed.
+enum { PB_K_FULL = 0, PB_K_EMPTY = 2, PB_V_FULL = 4, PB_V_EMPTY = 6, PB_Q_FULL = 8,
+       PB_S_FULL = 9, PB_P_READY = 11, PB_O_FINAL = 13, PB_DRAIN = 15, PB_COUNT = 16 };
 
 template <int D, int BLK, bool FP8>
 __global__ void __launch_bounds__(384, 1)
@@ -134,23 +137,43 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 for (int c = 0; c < C::NCH; ++c)
                     tma_load_3d(q_s + x * C::Q_BYTES + c * (128 * 128), &maps.q, &bars[PB_Q_FULL],
                                 c * C::CH, hk * G, s.q0 + t_begin + x * TOK);
-            int issued = 0;
-            for (int n = 0; n < n_items; ++n) {
-                const int st = n & 1;
-                if (n >= 2 && !mbar_wait(&bars[PB_KV_EMPTY + st], ((n - 2) >> 1) & 1, abort_flag,
-                                         kWaitLimitNs)) {
-                    set_error(p.err, kErrTimeout, kDetWaitBase + 0);
-                    break;
+            // K runs one item ahead of V: iteration n loads K(n), then V(n-1)
+            int k_issued = 0, v_issued = 0;
+            bool ok = true;
+            for (int n = 0; ok && n <= n_items; ++n) {
+                if (n < n_items) {
+                    const int st = n & 1;
+                    if (n >= 2 && !mbar_wait(&bars[PB_K_EMPTY + st], ((n - 2) >> 1) & 1,
+                                             abort_flag, kWaitLimitNs)) {
+                        set_error(p.err, kErrTimeout, kDetWaitBase + 0);
+                        ok = false;
+                        break;
+                    }
+                    issue_tile_load<D, BLK, FP8>(p, &maps.k, &maps.kb, s, b, hk, items[n],
+                                                 sbase + C::OFF_K + st * C::KV_BYTES,
+                                                 &bars[PB_K_FULL + st], true);
+                    ++k_issued;
                 }
-                issue_item_loads<D, BLK, FP8>(p, maps, s, b, hk, items[n],
-                                              sbase + C::OFF_K + st * C::KV_BYTES,
-                                              sbase + C::OFF_V + st * C::KV_BYTES,
-                                              &bars[PB_KV_FULL + st]);
-                ++issued;
+                if (n >= 1) {
+                    const int m = n - 1, st = m & 1;
+                    if (m >= 2 && !mbar_wait(&bars[PB_V_EMPTY + st], ((m - 2) >> 1) & 1,
+                                             abort_flag, kWaitLimitNs)) {
+                        set_error(p.err, kErrTimeout, kDetWaitBase + 0);
+                        ok = false;
+                        break;
+                    }
+                    issue_tile_load<D, BLK, FP8>(p, &maps.v, &maps.vb, s, b, hk, items[m],
+                                                 sbase + C::OFF_V + st * C::KV_BYTES,
+                                                 &bars[PB_V_FULL + st], true);
+                    ++v_issued;
+                }
             }
+            // never leave with copies in flight
             volatile int no_abort = 0;
-            for (int n = max(0, issued - 2); n < issued; ++n)
-                mbar_wait(&bars[PB_KV_FULL + (n & 1)], (n >> 1) & 1, &no_abort, kWaitLimitNs);
+            for (int n = max(0, k_issued - 2); n < k_issued; ++n)
+                mbar_wait(&bars[PB_K_FULL + (n & 1)], (n >> 1) & 1, &no_abort, kWaitLimitNs);
+            for (int n = max(0, v_issued - 2); n < v_issued; ++n)
+                mbar_wait(&bars[PB_V_FULL + (n & 1)], (n >> 1) & 1, &no_abort, kWaitLimitNs);
             mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, kWaitLimitNs);
       } else if (warp == 9 && lane == 0) {
         // -------------------------------------------------------------- MMA ---
@@ -163,7 +186,13 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             for (int n = 0; ok && n <= n_items; ++n) {
                 const int st = n & 1;
                 if (n < n_items &&
-                    !mbar_wait(&bars[PB_KV_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs)) {
+                    !mbar_wait(&bars[PB_K_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs)) {
+                    set_error(p.err, kErrTimeout, kDetWaitBase + 2);
+                    ok = false;
+                    break;
+                }
+                if (n >= 1 && !mbar_wait(&bars[PB_V_FULL + ((n - 1) & 1)], ((n - 1) >> 1) & 1,
+                                         abort_flag, kWaitLimitNs)) {
                     set_error(p.err, kErrTimeout, kDetWaitBase + 2);
                     ok = false;
                     break;
@@ -189,7 +218,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                             if constexpr (FP8) mma_f8_ts(o_tmem, p_tmem + ks * 8, bd, idesc_pv, acc);
                             else mma_bf16_ts(o_tmem, p_tmem + ks * 8, bd, idesc_pv, acc);
                         }
-                        if (x == 1) mma_commit(&bars[PB_KV_EMPTY + (m & 1)]);
+                        if (x == 1) mma_commit(&bars[PB_V_EMPTY + (m & 1)]);
                         if (m == n_items - 1) mma_commit(&bars[PB_O_FINAL + x]);
                     }
                     if (n < n_items) {
@@ -207,6 +236,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                             else mma_bf16_ss(s_tmem, ad, bd, idesc_qk, ks > 0);
                         }
                         mma_commit(&bars[PB_S_FULL + x]);
+                        if (x == 1) mma_commit(&bars[PB_K_EMPTY + st]);
                     }
                 }
             }
@@ -355,6 +385,14 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 tmem_st32(s_addr + c * 32, pk);
             }
             if (X == 0 && item >= 0 && item * BLK + BLK > s.Lk) {
+                // V(n) loads one step behind K(n): let it land before zeroing
+                // (V(n+2) cannot reuse the slot before this warpgroup's P(n))
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[PB_V_FULL + (n & 1)], (n >> 1) & 1,
+                                                       abort_flag, kWaitLimitNs))) {
+                    set_error(p.err, kErrTimeout, kDetWaitBase + 7);
+                    ok = false;
+                    break;
+                }
                 zero_v_tail<BLK, C::NCH>(smem + C::OFF_V + (n & 1) * C::KV_BYTES,
                                          max(0, s.Lk - item * BLK), r, 128);
                 fence_proxy_async_smem();

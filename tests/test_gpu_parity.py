@@ -266,3 +266,36 @@ def test_single_tile_kernel_on_large_groups(name, monkeypatch):
         ref, _, _ = H.oracle_out(inp, b, orc[b], keep)
         H.assert_close(H.out_seq(pr, inp, b).reshape(ref.shape), ref, inp.shape.dtype == "fp8",
                        f"{name} seq {b}")
+
+
+@pytest.mark.parametrize("boost,drop", [(6.0, 0.5), (40.0, None)])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_row_max_jumps_later_in_the_row(boost, drop, dtype):
+    """Keys of a later block scaled up so that, after the first kept blocks set
+    a row's reference maximum, a later block's logits exceed it by tens (x6)
+    or hundreds (x40) of log2 units: the attention kernel's rescale paths
+    (scale P down after the fact; redo the item from TMEM) must still match
+    the oracle.  The x40 case keeps every block (tau = +inf): a dropped block
+    with keys that large would turn the rounding of its mean (the MMA operand
+    of the correction) into logit errors of whole units, a different
+    question from the rescale paths tested here."""
+    shape = H.small_shape([1100], Hq=8, Hkv=2, dtype=dtype, seed=31)
+    inp = synth.make_inputs(shape)
+    # scale the stored K of block 5 (keeps the stored dtype; the oracle reads
+    # the same dequantised values)
+    blk = slice(5 * 128, 6 * 128)
+    kb = inp._kc[blk].float() * boost
+    if dtype == "fp8":
+        kb = kb.clamp(-448, 448)
+    inp._kc[blk] = kb.to(inp._kc.dtype)
+    orc = H.oracle_scores(inp)
+    tau = H.pick_tau(orc, drop) if drop is not None else float("inf")
+    pr = H.problem(inp, out_fill=float("nan"))
+    pr.prefill(tau)
+    pr.check()
+    keep = O.mask(orc[0][3], orc[0][4], tau)
+    assert keep[:, 6:, 5].mean() > 0.3  # the boosted block is kept by later rows
+    ref, _, _ = H.oracle_out(inp, 0, orc[0], keep)
+    got = H.out_seq(pr, inp, 0).reshape(ref.shape)
+    assert np.isfinite(got).all()
+    H.assert_close(got, ref, dtype == "fp8", f"boost {boost}")
