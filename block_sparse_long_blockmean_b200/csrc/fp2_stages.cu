@@ -150,7 +150,23 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
     const uint8_t* qrow = Q + (((size_t)(s.q0 + t0) * p.Hq + hk * G) * D) * ELT + (size_t)v * 16;
     const size_t tok_stride = (size_t)p.Hq * D * ELT;
-    for (int t = tg; t < n; t += TPP) {
+    // 8 loads in flight per thread before any is consumed
+    constexpr int U = 8;
+    int t = tg;
+    for (; t + (U - 1) * TPP < n; t += U * TPP) {
+        uint4 xs[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            xs[u] = __ldg(reinterpret_cast<const uint4*>(qrow + (size_t)(t + u * TPP) * tok_stride));
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float f[VEC];
+            unpack16<FP8>(xs[u], f);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] += f[e];
+        }
+    }
+    for (; t < n; t += TPP) {
         const uint4 x = __ldg(reinterpret_cast<const uint4*>(qrow + (size_t)t * tok_stride));
         float f[VEC];
         unpack16<FP8>(x, f);
@@ -180,32 +196,65 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
     const float* kb = p.kbar + ((size_t)b * p.Hkv + hk) * p.nkb_max * D + lane * PER_LANE;
     float* srow = p.scores + (((size_t)b * p.Hq + hk * G) * p.nqb_max + i) * p.nkb_max;
     const size_t head_stride = (size_t)p.nqb_max * p.nkb_max;
-    for (int j = warp; j <= iabs; j += 8) {
-        float kv[PER_LANE];
-        if constexpr (PER_LANE == 4) {
-            const float4 t = __ldg(reinterpret_cast<const float4*>(kb + (size_t)j * D));
-            kv[0] = t.x; kv[1] = t.y; kv[2] = t.z; kv[3] = t.w;
-        } else {
-            const float2 t = __ldg(reinterpret_cast<const float2*>(kb + (size_t)j * D));
-            kv[0] = t.x; kv[1] = t.y;
+    // Each warp takes 4 key blocks at a time: 4*G partial dot products per
+    // lane (lanes split d), summed over the warp by a reduce-scatter
+    // butterfly (each step halves the values a lane carries), so that the
+    // 4*G sums end up spread over the lanes instead of every lane holding all.
+    constexpr int NV = 4 * G;  // 4, 8, 16 or 32 values
+    for (int j0 = warp * 4; j0 <= iabs; j0 += 32) {
+        float v[NV];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int j = min(j0 + r, iabs);
+            float kv[PER_LANE];
+            if constexpr (PER_LANE == 4) {
+                const float4 t4 = __ldg(reinterpret_cast<const float4*>(kb + (size_t)j * D));
+                kv[0] = t4.x; kv[1] = t4.y; kv[2] = t4.z; kv[3] = t4.w;
+            } else {
+                const float2 t2 = __ldg(reinterpret_cast<const float2*>(kb + (size_t)j * D));
+                kv[0] = t2.x; kv[1] = t2.y;
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < PER_LANE; ++e) a = fmaf(qv[g][e], kv[e], a);
+                v[r * G + g] = a;
+            }
         }
-        float dot[G];
+        // reduce-scatter: after the step with offset o (o = 16, 8, ...), a lane
+        // keeps the half of its values selected by its bit o and adds the
+        // partner's copy of that half
+        int nv = NV;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float a = 0.f;
+        for (int o = 16; o >= 1; o >>= 1) {
+            if (nv > 1) {
+                const bool upper = (lane & o) != 0;
+                const int half = nv >> 1;
 #pragma unroll
-            for (int e = 0; e < PER_LANE; ++e) a = fmaf(qv[g][e], kv[e], a);
-            dot[g] = a;
+                for (int x = 0; x < NV / 2; ++x) {
+                    if (x < half) {
+                        const float send = upper ? v[x] : v[x + half];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+                        v[x] = (upper ? v[x + half] : v[x]) + recv;
+                    }
+                }
+                nv = half;
+            } else {
+                v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+            }
         }
+        // lane holds value index = bits of (lane >> (5 - log2 NV)) selected
+        // above: value idx = sum over steps of (upper ? half : 0)
+        int idx = 0, h = NV >> 1;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-            for (int g = 0; g < G; ++g) dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
-        if (lane < G) {
-            float mine = dot[0];
-#pragma unroll
-            for (int g = 1; g < G; ++g) if (lane == g) mine = dot[g];
-            srow[(size_t)lane * head_stride + j] = mine * scale;
+        for (int o = 16; o >= 1 && h >= 1; o >>= 1, h >>= 1)
+            if (lane & o) idx += h;
+        constexpr int COPIES = 32 / NV;  // lanes holding the same value
+        if ((lane & (COPIES - 1)) == 0) {
+            const int r = idx / G, g = idx % G;
+            const int j = j0 + r;
+            if (j <= iabs) srow[(size_t)g * head_stride + j] = v[0] * scale;
         }
     }
 }
