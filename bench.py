@@ -47,6 +47,38 @@ def parse():
     return ap.parse_args()
 
 
+ATTN_SOURCES = ["fp2_attn_pair.cu", "fp2_attn.cu", "fp2_attn_common.cuh", "fp2_device.cuh",
+                "fp2_seq.cuh", "fp2_internal.h", "fp2_exp2_poly.h"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_pair_128k_traffic.md")
+
+
+def attn_source_hash() -> str:
+    """sha256 (12 hex) over the attention kernel's sources: ties a recorded ncu
+    traffic figure to the exact kernel it was taken on."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_long_blockmean_b200", "csrc")
+    for f in ATTN_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(dtype: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when the summary was taken on a different kernel source."""
+    try:
+        txt = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    import re
+    m = re.search(r"source_sha:\s*([0-9a-f]{12})", txt)
+    t = re.search(rf"dram_bytes_per_launch_{dtype}:\s*([0-9.eE+]+)", txt)
+    if not m or not t or m.group(1) != attn_source_hash():
+        return None
+    return float(t.group(1))
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -443,7 +475,7 @@ def main():
                    "l2": "inputs (1.6 GB) larger than L2; no flush",
                    "per_gpu": "one independent layer per GPU"},
         "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
-                     "frac": eff / peak, "traffic": None,
+                     "frac": eff / peak, "traffic": recorded_traffic(main_dt),
                      "kernel": "fp2_attn (attn_kernel)",
                      "peak_source": f"{peak_src} bf16_tflops_sustained" +
                                     (" x2 (fp8/bf16 nominal ratio)" if main_dt == "fp8" else "")},
