@@ -37,10 +37,12 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="fp2", choices=["fp2", "reference"])
     ap.add_argument("--dtype", default="both", choices=["bf16", "fp8", "both"])
-    ap.add_argument("--drop", type=float, default=DROP)
-    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[2, 3],
+    ap.add_argument("--drop", type=float, default=None,
+                    help="target dropped fraction (default: the workload's, 0.8 at 128K)")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[2, 3, 5],
                     help="3 = the 128K layer (the metric's workload); 2 = the 32K layer, a "
-                         "smaller case for profiler captures")
+                         "smaller case for profiler captures; 5 = a 32K chunk on a "
+                         "229376-token paged prefix (also times the block-mean cache)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -208,25 +210,27 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
     v = inp.v.to(dev)
     cu = inp.cu_seqlens_q.to(dev)
     lk = inp.seqlens_k.to(dev)
-    cuk = inp.cu_seqlens_k.to(dev)
+    pt = inp.page_table.to(dev) if inp.paged else None
+    cuk = None if inp.paged else inp.cu_seqlens_k.to(dev)
     sc = [x.to(dev) if x is not None else None for x in (inp.q_scale, inp.k_scale, inp.v_scale)]
     stream = torch.cuda.Stream(dev)
     pr = fp2.make_problem(q, k, v, cu, Hq=s.Hq, Hkv=s.Hkv, d=s.d, block=s.B, dtype=dt,
                           max_seqlen_q=max(s.lens_q), max_seqlen_k=max(s.lens_k),
-                          seqlens_k=lk, cu_seqlens_k=cuk, q_scale=sc[0], k_scale=sc[1],
-                          v_scale=sc[2], stream=stream.cuda_stream)
+                          seqlens_k=lk, cu_seqlens_k=cuk, page_table=pt,
+                          page_size=k.shape[1] if inp.paged else 0, q_scale=sc[0],
+                          k_scale=sc[1], v_scale=sc[2], stream=stream.cuda_stream)
     P = pr.params
     B = s.B
     with torch.cuda.stream(stream):
         # tau for the target drop, from this GPU's own scores (not timed)
-        fp2.blockmean(k, v, None, cu, B, dt, P)
+        fp2.blockmean(k, v, pt, cu, B, dt, P)
         fp2.score(q, cu, B, dt, P)
-        tau = fp2.calibrate_tau(cu, B, args.drop, P)
+        tau = fp2.calibrate_tau(cu, B, args.drop if args.drop is not None else s.drop, P)
 
         def step(ev=None):
             if ev is not None:
                 ev[0].record(stream)
-            fp2.blockmean(k, v, None, cu, B, dt, P)
+            fp2.blockmean(k, v, pt, cu, B, dt, P)
             if ev is not None:
                 ev[1].record(stream)
             fp2.score(q, cu, B, dt, P)
@@ -235,7 +239,7 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
             fp2.mask(cu, tau, B, P)
             if ev is not None:
                 ev[3].record(stream)
-            fp2.attn(q, k, v, None, cu, None, B, dt, pr.out, P)
+            fp2.attn(q, k, v, pt, cu, None, B, dt, pr.out, P)
             if ev is not None:
                 ev[4].record(stream)
 
@@ -275,9 +279,9 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
         if not args.no_dense:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             fp2.mask(cu, math.inf, B, P)
-            fp2.attn(q, k, v, None, cu, None, B, dt, pr.out, P)  # warm
+            fp2.attn(q, k, v, pt, cu, None, B, dt, pr.out, P)  # warm
             e0.record(stream)
-            fp2.attn(q, k, v, None, cu, None, B, dt, pr.out, P)
+            fp2.attn(q, k, v, pt, cu, None, B, dt, pr.out, P)
             e1.record(stream)
             stream.synchronize()
             dense = {"attn_ms": e0.elapsed_time(e1),
@@ -289,8 +293,8 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
             # through the public API with HOST buffers: H2D of q, k, v from
             # pinned memory, fp2_prefill, D2H of the output, every step
             hq = inp.q.pin_memory()
-            hk = inp._kc.pin_memory()
-            hv = inp._vc.pin_memory()
+            hk = inp.k.pin_memory()
+            hv = inp.v.pin_memory()
             hout = torch.empty(pr.out.shape, dtype=torch.bfloat16).pin_memory()
             nsteps = max(2, min(args.steps, 5))
             for it in range(nsteps + 1):
@@ -300,7 +304,7 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
                 q.copy_(hq, non_blocking=True)
                 k.copy_(hk, non_blocking=True)
                 v.copy_(hv, non_blocking=True)
-                fp2.prefill(q, k, v, None, cu, tau, B, dt, pr.out, P)
+                fp2.prefill(q, k, v, pt, cu, tau, B, dt, pr.out, P)
                 hout.copy_(pr.out, non_blocking=True)
             eb.record(stream)
             stream.synchronize()
@@ -311,8 +315,51 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
                                              hk.numel() * hk.element_size() +
                                              hv.numel() * hv.element_size()),
                    "d2h_bytes_per_step": int(hout.numel() * hout.element_size())}
+        mean_cache = None
+        prefixes = [Lk - Lq for Lq, Lk in zip(s.lens_q, s.lens_k)]
+        if inp.paged and max(prefixes) > 0:
+            # step 1 with the block-mean cache: fill it as the earlier chunks
+            # would have (the whole sequence as one chunk), then time the
+            # current chunk's step 1 against the plain one
+            nblk = [-(-Lk // B) for Lk in s.lens_k]
+            slots = sum(nblk)
+            table = torch.full((len(nblk), max(nblk)), -1, dtype=torch.int32)
+            off = 0
+            for b, n in enumerate(nblk):
+                table[b, :n] = torch.arange(off, off + n, dtype=torch.int32)
+                off += n
+            table = table.to(dev)
+            cache = torch.empty((slots, 2, s.Hkv, s.d), dtype=torch.float32, device=dev)
+            cu_full = torch.tensor(np.concatenate([[0], np.cumsum(s.lens_k)]), dtype=torch.int32,
+                                   device=dev)
+            fill = fp2.make_problem(q, k, v, cu_full, Hq=s.Hq, Hkv=s.Hkv, d=s.d, block=B, dtype=dt,
+                                    max_seqlen_q=max(s.lens_k), max_seqlen_k=max(s.lens_k),
+                                    seqlens_k=lk, page_table=pt, page_size=k.shape[1],
+                                    q_scale=sc[0], k_scale=sc[1], v_scale=sc[2],
+                                    stream=stream.cuda_stream)
+            fill.params.total_q = int(sum(s.lens_k))
+            fp2.blockmean_cached(k, v, pt, cu_full, table, max(nblk), cache, slots, B, dt,
+                                 fill.params)
+            fill.check()
+            del fill
+            t_plain, t_cached = [], []
+            for it in range(6):
+                ea, eb, ec = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                ea.record(stream)
+                fp2.blockmean(k, v, pt, cu, B, dt, P)
+                eb.record(stream)
+                fp2.blockmean_cached(k, v, pt, cu, table, max(nblk), cache, slots, B, dt, P)
+                ec.record(stream)
+                stream.synchronize()
+                if it:
+                    t_plain.append(ea.elapsed_time(eb))
+                    t_cached.append(eb.elapsed_time(ec))
+            pr.check()
+            mean_cache = {"blockmean_ms": float(np.median(t_plain)),
+                          "blockmean_cached_ms": float(np.median(t_cached)),
+                          "prefix_blocks_from_cache": int(sum(p_ // B for p_ in prefixes))}
     res = {
-        "dtype": dtype_name, "tau": tau, "drop_fraction": drop_frac,
+        "dtype": dtype_name, "tau": tau, "drop_fraction": drop_frac, "mean_cache": mean_cache,
         "total_ms": total_ms, "ms_per_step": total_ms / args.steps,
         "stage_ms": {"blockmean": stage_ms[0], "score": stage_ms[1], "mask": stage_ms[2],
                      "attn": stage_ms[3]},
@@ -336,21 +383,22 @@ def cpu_baseline(inp, tau, budget_blocks=4, heads_per_block=8):
     K, V = inp.seq_k(0), inp.seq_v(0)
     kbar, vbar, cnt = O.blockmean(K, V, B)
     Lq = s.lens_q[0]
+    pb = (s.lens_k[0] - Lq) // B
     nqb = -(-Lq // B)
     parts = []
     for i0 in range(0, nqb, 64):
         Qc = inp._deq(inp.q[i0 * B: min(Lq, (i0 + 64) * B)], inp.q_scale)
         parts.append(O.pool_q(Qc, B))
     qbar = np.concatenate(parts, axis=1)
-    S = O.score(qbar, kbar, 0)
-    keep = O.mask(S, 0, tau)
+    S = O.score(qbar, kbar, pb)
+    keep = O.mask(S, pb, tau)
     t_sel = time.time() - t0
     blocks = [int((m + 0.5) * nqb / budget_blocks) for m in range(budget_blocks)]
     heads = np.arange(heads_per_block, dtype=np.int32)
     t1 = time.time()
     for i in blocks:
         Qb = inp._deq(inp.q[i * B: min(Lq, (i + 1) * B)], inp.q_scale)
-        O.attn_query_block(Qb, K, V, kbar, vbar, cnt, keep[:, i], B, i, heads)
+        O.attn_query_block(Qb, K, V, kbar, vbar, cnt, keep[:, i], B, pb + i, heads)
     t_attn = time.time() - t1
     scale = (nqb / budget_blocks) * (s.Hq / heads_per_block)
     est_s = t_sel + t_attn * scale
@@ -378,7 +426,7 @@ def reference_arm(args):
     for i0 in range(0, nqb, 64):
         parts.append(O.pool_q(inp._deq(inp.q[i0 * B: (i0 + 64) * B], None), B))
     S = O.score(np.concatenate(parts, axis=1), kbar, 0)
-    tau = O.tau_for_drop([S], [0], args.drop)
+    tau = O.tau_for_drop([S], [0], args.drop if args.drop is not None else shape.drop)
     keep = O.mask(S, 0, tau)
     rng = np.random.default_rng(0)
     times = []
@@ -399,7 +447,8 @@ def reference_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": synth.WORKLOAD_NAMES[args.workload], "drop": args.drop},
+            "config": {"workload": synth.WORKLOAD_NAMES[args.workload],
+                       "drop": args.drop if args.drop is not None else shape.drop},
             "cpu_baseline": {"value": ms, "unit": "ms/layer", "cores": O.num_threads(),
                              "kind": "oracle",
                              "sample": "per step: corrected attention of 4 heads x 1 random "
@@ -455,6 +504,8 @@ def main():
                "tensor_frac_executed_measured": eff * x["union_inflation"] / peak,
                "stage_ms": x["stage_ms"],
                "prefill_roofline_frac": (x["kept_flops"] / peak / 1e12) / (x["ms_per_step"] * 1e-3)}
+        if x.get("mean_cache"):
+            out["mean_cache"] = x["mean_cache"]
         if x["dense"]:
             out["dense_attn_ms"] = x["dense"]["attn_ms"]
             out["dense_tflops"] = x["dense"]["tflops"]
@@ -471,7 +522,10 @@ def main():
         "config": {"workload": synth.WORKLOAD_NAMES[args.workload],
                    "seq_len": synth.workload(args.workload).lens_q[0],
                    "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128, "block": 128,
-                   "target_drop": args.drop, "layout": "contiguous K/V",
+                   "target_drop": args.drop if args.drop is not None else
+                   synth.workload(args.workload).drop,
+                   "layout": "paged K/V (64-token pages)" if synth.workload(args.workload).page_size
+                   else "contiguous K/V",
                    "l2": "inputs (1.6 GB) larger than L2; no flush",
                    "per_gpu": "one independent layer per GPU"},
         "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",

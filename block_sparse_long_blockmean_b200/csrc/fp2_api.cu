@@ -183,6 +183,34 @@ fp2_status fp2_blockmean(const void* k_cache, const void* v_cache, const int32_t
     return cuda_status(fp2::launch_blockmean(kp, k_cache, v_cache, stream_of(params)));
 }
 
+static fp2_status attach_mean_cache(KParams& kp, const int32_t* block_table,
+                                    int max_blocks_per_seq, float* mean_cache, int num_slots) {
+    if (!block_table || !mean_cache || max_blocks_per_seq < 1 || num_slots < 1)
+        return FP2_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(mean_cache) & 15u) != 0) return FP2_ERR_INVALID_ARG;
+    kp.mean_cache = mean_cache;
+    kp.block_table = block_table;
+    kp.max_blocks = max_blocks_per_seq;
+    kp.num_slots = num_slots;
+    return FP2_OK;
+}
+
+fp2_status fp2_blockmean_cached(const void* k_cache, const void* v_cache,
+                                const int32_t* page_table, const int32_t* cu_seqlens,
+                                const int32_t* block_table, int max_blocks_per_seq,
+                                float* mean_cache, int num_slots, int block, fp2_dtype dtype,
+                                const fp2_params* params) {
+    KParams kp;
+    fp2_status st = prepare(params, block, dtype, cu_seqlens, page_table, kp);
+    if (st != FP2_OK) return st;
+    if (!k_cache || !v_cache) return FP2_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return FP2_ERR_INVALID_ARG;
+    if ((st = attach_mean_cache(kp, block_table, max_blocks_per_seq, mean_cache, num_slots)) !=
+        FP2_OK)
+        return st;
+    return cuda_status(fp2::launch_blockmean(kp, k_cache, v_cache, stream_of(params)));
+}
+
 fp2_status fp2_score(const void* q, const int32_t* cu_seqlens, int block, fp2_dtype dtype,
                      const fp2_params* params) {
     KParams kp;
@@ -218,12 +246,18 @@ fp2_status fp2_attn(const void* q, const void* k_cache, const void* v_cache,
     return cuda_status(e);
 }
 
-fp2_status fp2_prefill(const void* q, const void* k_cache, const void* v_cache,
-                       const int32_t* page_table, const int32_t* cu_seqlens, float tau,
-                       int block, fp2_dtype dtype, void* out, const fp2_params* params) {
+static fp2_status prefill_impl(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* page_table, const int32_t* cu_seqlens, float tau,
+                               int block, fp2_dtype dtype, void* out, const fp2_params* params,
+                               const int32_t* block_table, int max_blocks_per_seq,
+                               float* mean_cache, int num_slots) {
     KParams kp;
     fp2_status st = prepare(params, block, dtype, cu_seqlens, page_table, kp);
     if (st != FP2_OK) return st;
+    if (mean_cache &&
+        (st = attach_mean_cache(kp, block_table, max_blocks_per_seq, mean_cache, num_slots)) !=
+            FP2_OK)
+        return st;
     if (!q || !k_cache || !v_cache || !out) return FP2_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return FP2_ERR_INVALID_ARG;
@@ -232,11 +266,29 @@ fp2_status fp2_prefill(const void* q, const void* k_cache, const void* v_cache,
     if (!page_table && kp.total_k == 0) return FP2_ERR_INVALID_ARG;
     cudaStream_t s = stream_of(params);
     cudaError_t e = fp2::launch_blockmean(kp, k_cache, v_cache, s);
+    kp.mean_cache = nullptr;  // only the block means use the cache
     if (e == cudaSuccess) e = fp2::launch_score(kp, q, s);
     if (e == cudaSuccess) e = fp2::launch_mask(kp, tau, s);
     if (e == cudaSuccess) e = fp2::launch_attn(kp, q, k_cache, v_cache, kp.kept_bits, out, s);
     if (e == cudaErrorInvalidValue) return FP2_ERR_UNSUPPORTED;
     return cuda_status(e);
+}
+
+fp2_status fp2_prefill(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* page_table, const int32_t* cu_seqlens, float tau,
+                       int block, fp2_dtype dtype, void* out, const fp2_params* params) {
+    return prefill_impl(q, k_cache, v_cache, page_table, cu_seqlens, tau, block, dtype, out,
+                        params, nullptr, 0, nullptr, 0);
+}
+
+fp2_status fp2_prefill_cached(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* page_table, const int32_t* cu_seqlens, float tau,
+                              int block, fp2_dtype dtype, void* out, const fp2_params* params,
+                              const int32_t* block_table, int max_blocks_per_seq,
+                              float* mean_cache, int num_slots) {
+    if (!mean_cache) return FP2_ERR_INVALID_ARG;
+    return prefill_impl(q, k_cache, v_cache, page_table, cu_seqlens, tau, block, dtype, out,
+                        params, block_table, max_blocks_per_seq, mean_cache, num_slots);
 }
 
 fp2_status fp2_workspace_init(const fp2_params* params) {

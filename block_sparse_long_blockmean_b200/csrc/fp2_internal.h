@@ -33,6 +33,12 @@ struct KParams {
     int32_t* kept_idx;         // [S][Hq][nqb_max][nkb_max]
     int32_t* kept_cnt;         // [S][Hq][nqb_max]
     uint32_t* kept_bits;       // [S][Hq][nqb_max][nw]
+    // optional block-mean cache (chunked prefill): raw means of the stored
+    // K and V values, [num_slots][2][Hkv][d] fp32, slot of (b, j) in
+    // block_table[b * max_blocks + j]
+    float* mean_cache;
+    const int32_t* block_table;
+    int max_blocks, num_slots;
 };
 
 // Detail codes stored beside an error code.
@@ -40,6 +46,7 @@ enum : uint32_t {
     kDetSeqLen = 1,      // Lq or Lk outside [0, max_seqlen_*] or Lk < Lq
     kDetPrefix = 2,      // (Lk - Lq) % block != 0
     kDetPage = 3,        // page id outside [0, num_pages)
+    kDetSlot = 4,        // block-mean cache slot outside [0, num_slots) or beyond max_blocks
     kDetWaitBase = 16,   // + pipeline wait site
 };
 

@@ -72,6 +72,35 @@ __global__ void __launch_bounds__(128) blockmean_kernel(KParams p, const uint8_t
     }
     const int t0 = j * p.B;
     const int n = min(p.B, s.Lk - t0);
+    // block-mean cache: blocks wholly inside the resident prefix are read
+    // from it, the others are computed and written back
+    float* slot_ptr = nullptr;
+    if (p.mean_cache) {
+        const int slot = j < p.max_blocks ? p.block_table[(size_t)b * p.max_blocks + j] : -1;
+        if (slot < 0 || slot >= p.num_slots) {
+            set_error(p.err, kErrBounds, kDetSlot);
+            return;
+        }
+        slot_ptr = p.mean_cache + ((size_t)slot * 2 * p.Hkv + hk) * D;
+    }
+    const float ks = FP8 ? p.k_scale[hk] : 1.f;
+    const float vs = FP8 ? p.v_scale[hk] : 1.f;
+    auto emit = [&](int c, float mk, float mv) {  // mk, mv: means of the stored values
+        p.kbar[orow + c] = mk * ks;                // dequantised
+        p.vbar[orow + c] = mv * vs;
+        if constexpr (FP8) {
+            reinterpret_cast<__nv_fp8_e4m3*>(p.kbar_op)[orow + c] = __nv_fp8_e4m3(mk);
+            reinterpret_cast<__nv_fp8_e4m3*>(p.vbar_op)[orow + c] = __nv_fp8_e4m3(mv);
+        } else {
+            reinterpret_cast<__nv_bfloat16*>(p.kbar_op)[orow + c] = __float2bfloat16(mk);
+            reinterpret_cast<__nv_bfloat16*>(p.vbar_op)[orow + c] = __float2bfloat16(mv);
+        }
+    };
+    if (slot_ptr && t0 + p.B <= s.P) {
+        for (int c = threadIdx.x; c < D; c += 128)
+            emit(c, slot_ptr[c], slot_ptr[(size_t)p.Hkv * D + c]);
+        return;
+    }
     const int lv = threadIdx.x % TPR, rg = threadIdx.x / TPR;
     float ak[VEC], av[VEC];
 #pragma unroll
@@ -98,8 +127,6 @@ __global__ void __launch_bounds__(128) blockmean_kernel(KParams p, const uint8_t
     }
     __syncthreads();
     const float inv = 1.f / (float)n;
-    const float ks = FP8 ? p.k_scale[hk] : 1.f;
-    const float vs = FP8 ? p.v_scale[hk] : 1.f;
     for (int c = threadIdx.x; c < D; c += 128) {
         float sk = 0.f, sv = 0.f;
 #pragma unroll
@@ -107,15 +134,11 @@ __global__ void __launch_bounds__(128) blockmean_kernel(KParams p, const uint8_t
             sk += red[0][r][c];
             sv += red[1][r][c];
         }
-        const float mk = sk * inv, mv = sv * inv;  // mean of the stored values
-        p.kbar[orow + c] = mk * ks;                // dequantised
-        p.vbar[orow + c] = mv * vs;
-        if constexpr (FP8) {
-            reinterpret_cast<__nv_fp8_e4m3*>(p.kbar_op)[orow + c] = __nv_fp8_e4m3(mk);
-            reinterpret_cast<__nv_fp8_e4m3*>(p.vbar_op)[orow + c] = __nv_fp8_e4m3(mv);
-        } else {
-            reinterpret_cast<__nv_bfloat16*>(p.kbar_op)[orow + c] = __float2bfloat16(mk);
-            reinterpret_cast<__nv_bfloat16*>(p.vbar_op)[orow + c] = __float2bfloat16(mv);
+        const float mk = sk * inv, mv = sv * inv;
+        emit(c, mk, mv);
+        if (slot_ptr) {
+            slot_ptr[c] = mk;
+            slot_ptr[(size_t)p.Hkv * D + c] = mv;
         }
     }
 }

@@ -90,7 +90,12 @@ SIGNATURES = {
                                    ctypes.c_int, _VP, _PP]),
     "fp2_prefill_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, ctypes.c_float, ctypes.c_int,
                                            ctypes.c_int, _VP, _PP]),
+    "fp2_prefill_cached": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, ctypes.c_float, ctypes.c_int,
+                                          ctypes.c_int, _VP, _PP, _VP, ctypes.c_int, _VP,
+                                          ctypes.c_int]),
     "fp2_blockmean": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, ctypes.c_int, _PP]),
+    "fp2_blockmean_cached": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, ctypes.c_int, _VP,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, _PP]),
     "fp2_score": (ctypes.c_int, [_VP, _VP, ctypes.c_int, ctypes.c_int, _PP]),
     "fp2_mask": (ctypes.c_int, [_VP, ctypes.c_float, ctypes.c_int, _PP]),
     "fp2_attn": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int, ctypes.c_int, _VP,
@@ -172,6 +177,24 @@ def blockmean(k_cache, v_cache, page_table, cu_seqlens, block: int, dtype: int,
               params: Params) -> None:
     _check(lib().fp2_blockmean(_ptr(k_cache), _ptr(v_cache), _ptr(page_table), _ptr(cu_seqlens),
                                block, dtype, ctypes.byref(params)), "fp2_blockmean")
+
+
+def prefill_cached(q, k_cache, v_cache, page_table, cu_seqlens, tau: float, block: int,
+                   dtype: int, out, params: Params, block_table, max_blocks_per_seq: int,
+                   mean_cache, num_slots: int) -> None:
+    _check(lib().fp2_prefill_cached(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                                    _ptr(cu_seqlens), float(tau), block, dtype, _ptr(out),
+                                    ctypes.byref(params), _ptr(block_table), max_blocks_per_seq,
+                                    _ptr(mean_cache), num_slots), "fp2_prefill_cached")
+
+
+def blockmean_cached(k_cache, v_cache, page_table, cu_seqlens, block_table,
+                     max_blocks_per_seq: int, mean_cache, num_slots: int, block: int, dtype: int,
+                     params: Params) -> None:
+    _check(lib().fp2_blockmean_cached(_ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                                      _ptr(cu_seqlens), _ptr(block_table), max_blocks_per_seq,
+                                      _ptr(mean_cache), num_slots, block, dtype,
+                                      ctypes.byref(params)), "fp2_blockmean_cached")
 
 
 def score(q, cu_seqlens, block: int, dtype: int, params: Params) -> None:

@@ -130,12 +130,38 @@ fp2_status fp2_prefill(const void* q, const void* k_cache, const void* v_cache,
                        float tau, int block, fp2_dtype dtype, void* out,
                        const fp2_params* params);
 
+/* fp2_prefill with step 1 served by the block-mean cache (fp2_blockmean_cached). */
+fp2_status fp2_prefill_cached(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* page_table, const int32_t* cu_seqlens, float tau,
+                              int block, fp2_dtype dtype, void* out, const fp2_params* params,
+                              const int32_t* block_table, int max_blocks_per_seq,
+                              float* mean_cache, int num_slots);
+
 /* Step 1 (explainer section 2.1, the mean of the dropped tokens): block means
  * of K and V into the workspace (kbar, vbar, kbar_op, vbar_op); key blocks
  * beyond a sequence's end are written as zeros. */
 fp2_status fp2_blockmean(const void* k_cache, const void* v_cache, const int32_t* page_table,
                          const int32_t* cu_seqlens, int block, fp2_dtype dtype,
                          const fp2_params* params);
+
+/* Step 1 for a chunked prefill over a resident prefix, with a block-mean
+ * cache kept beside the paged KV cache (so a new chunk does not re-read the
+ * whole prefix to average it).  The cache is caller-owned device memory,
+ * mean_cache fp32 [num_slots][2][Hkv][d]: per slot the means of the STORED
+ * K values, then of the stored V values, of one key block (before any FP8
+ * scale).  block_table int32 [num_seqs][max_blocks_per_seq] (device) gives
+ * the slot of key block j of sequence b.  Blocks wholly inside the prefix
+ * (j*block + block <= Lk - Lq) are read from their slot; every other block of
+ * the sequence is averaged from k_cache/v_cache and ALSO written to its slot
+ * (so the next chunk finds it).  The workspace receives exactly what
+ * fp2_blockmean would write.  A slot id outside [0, num_slots) or a block
+ * beyond max_blocks_per_seq records FP2_ERR_DEVICE_BOUNDS (detail 4).
+ * mean_cache must be 16-byte aligned. */
+fp2_status fp2_blockmean_cached(const void* k_cache, const void* v_cache,
+                                const int32_t* page_table, const int32_t* cu_seqlens,
+                                const int32_t* block_table, int max_blocks_per_seq,
+                                float* mean_cache, int num_slots, int block, fp2_dtype dtype,
+                                const fp2_params* params);
 
 /* Step 2 (abstract: instantaneous pattern discovery): pools each query block
  * (mean of its valid rows) and writes s_ij = qbar_i . kbar_j / sqrt(d) for
