@@ -54,7 +54,8 @@ struct AttnCfg {
     static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
     static constexpr int OFF_BAR = OFF_P + P_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + 256;
-    static constexpr int OFF_ITEMS = OFF_MISC + 64;
+    static constexpr int OFF_RING = OFF_MISC + 64;  // page ids of upcoming items
+    static constexpr int OFF_ITEMS = OFF_RING + kPageRing * kMaxBoxes * 4;
     static_assert(NCH >= 1 && PCH >= 1, "tile shape");
     static_assert(D % 32 == 0 && BLK % 32 == 0, "tile shape");
 };
@@ -130,6 +131,9 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     if (warp == 0) {
         // ------------------------------------------------------ producer ---
+        // the whole warp resolves page ids 32 items at a time; lane 0 waits
+        // and issues every copy
+        int* pring = reinterpret_cast<int*>(smem + C::OFF_RING);
         if (lane == 0) {
             prefetch_tmap(&maps.q);
             prefetch_tmap(&maps.k);
@@ -138,30 +142,35 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             for (int c = 0; c < C::NCH; ++c)
                 tma_load_3d(q_s + c * (128 * 128), &maps.q, &bars[B_Q_FULL], c * C::CH, hk * G,
                             s.q0 + t_begin);
-            int issued = 0;
-            for (int n = 0; n < n_items; ++n) {
+        }
+        int issued = 0;
+        bool ok = true;
+        for (int n = 0; n < n_items; ++n) {
+            if (n % 32 == 0) fill_page_ring<BLK>(p, s, b, items, n_items, n, pring);
+            if (lane == 0) {
                 const int st = n & 1;
                 if (n >= 2 && !mbar_wait(&bars[B_KV_EMPTY + st], ((n - 2) >> 1) & 1, abort_flag,
                                          kWaitLimitNs)) {
                     set_error(p.err, kErrTimeout, kDetWaitBase + 0);
-                    break;
+                    ok = false;
+                } else {
+                    issue_item_loads<D, BLK, FP8>(p, maps, s, b, hk, items[n],
+                                                  pring + (n % kPageRing) * kMaxBoxes,
+                                                  sbase + C::OFF_K + st * C::KV_BYTES,
+                                                  sbase + C::OFF_V + st * C::KV_BYTES,
+                                                  &bars[B_KV_FULL + st]);
+                    ++issued;
                 }
-                issue_item_loads<D, BLK, FP8>(p, maps, s, b, hk, items[n],
-                                              sbase + C::OFF_K + st * C::KV_BYTES,
-                                              sbase + C::OFF_V + st * C::KV_BYTES,
-                                              &bars[B_KV_FULL + st]);
-                ++issued;
             }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        }
+        if (lane == 0) {
             // never leave with copies in flight: wait (bounded) for the loads
             // of the last two stages, whatever happened above
-            for (int n = max(0, issued - 2); n < issued; ++n) {
-                volatile int no_abort = 0;
+            volatile int no_abort = 0;
+            for (int n = max(0, issued - 2); n < issued; ++n)
                 mbar_wait(&bars[B_KV_FULL + (n & 1)], (n >> 1) & 1, &no_abort, kWaitLimitNs);
-            }
-            {
-                volatile int no_abort = 0;
-                mbar_wait(&bars[B_Q_FULL], 0, &no_abort, kWaitLimitNs);
-            }
+            mbar_wait(&bars[B_Q_FULL], 0, &no_abort, kWaitLimitNs);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issue ---

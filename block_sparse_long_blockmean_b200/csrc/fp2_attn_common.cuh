@@ -101,8 +101,8 @@ __device__ __forceinline__ int build_items(int G, int iabs, int nw_c, const uint
 template <int D, int BLK, bool FP8>
 __device__ __forceinline__ void issue_tile_load(const KParams& p, const CUtensorMap* map,
                                                 const CUtensorMap* mean_map, const SeqInfo& s,
-                                                int b, int hk, int item, uint32_t dst,
-                                                uint64_t* full, bool arrive) {
+                                                int b, int hk, int item, const int* pages,
+                                                uint32_t dst, uint64_t* full, bool arrive) {
     constexpr int ELT = FP8 ? 1 : 2;
     constexpr int CH = 128 / ELT;
     constexpr int NCH = D / CH;
@@ -116,22 +116,11 @@ __device__ __forceinline__ void issue_tile_load(const KParams& p, const CUtensor
             for (int c = 0; c < NCH; ++c)
                 tma_load_3d(dst + c * BLK * 128, map, full, c * CH, hk, s.k0 + j * BLK);
         } else {
+            // pages[sb]: physical page of rows [sb*R, sb*R+R) of the block, or
+            // -1 (past the sequence end / invalid id: not loaded)
             const int R = min(p.page_size, BLK);
             int nbox = 0;
-            int pages[BLK / 16];
-            for (int sb = 0; sb < BLK / R; ++sb) {
-                const int tok = j * BLK + sb * R;
-                int pg = -1;
-                if (tok < s.Lk) {
-                    pg = p.page_table[(size_t)b * p.max_pages + tok / p.page_size];
-                    if (pg < 0 || pg >= p.num_pages) {
-                        set_error(p.err, kErrBounds, kDetPage);
-                        pg = -1;
-                    }
-                }
-                pages[sb] = pg;
-                nbox += (pg >= 0);
-            }
+            for (int sb = 0; sb < BLK / R; ++sb) nbox += (pages[sb] >= 0);
             if (arrive) mbar_arrive_expect_tx(full, (uint32_t)(nbox * NCH * R * 128));
             else mbar_expect_tx(full, (uint32_t)(nbox * NCH * R * 128));
             for (int sb = 0; sb < BLK / R; ++sb) {
@@ -153,14 +142,47 @@ __device__ __forceinline__ void issue_tile_load(const KParams& p, const CUtensor
     }
 }
 
+// Page ids of the work items are resolved by the whole producer warp, 32
+// items at a time (one lane per item), into a ring of kPageRing items x
+// kMaxBoxes sub-boxes in shared memory: the issuing lane then reads them from
+// shared memory instead of making one dependent page-table load per tile.
+constexpr int kPageRing = 64;
+constexpr int kMaxBoxes = 8;  // BLK / page_size for page_size >= 16, BLK <= 128
+
+template <int BLK>
+__device__ __forceinline__ void fill_page_ring(const KParams& p, const SeqInfo& s, int b,
+                                               const int* items, int n_items, int n0, int* ring) {
+    const int lane = threadIdx.x & 31;
+    const int n = n0 + lane;
+    if (p.paged && n < n_items && items[n] >= 0) {
+        const int j = items[n];
+        const int R = min(p.page_size, BLK);
+        int* dst = ring + (n % kPageRing) * kMaxBoxes;
+        for (int sb = 0; sb < BLK / R; ++sb) {
+            const int tok = j * BLK + sb * R;
+            int pg = -1;
+            if (tok < s.Lk) {
+                pg = p.page_table[(size_t)b * p.max_pages + tok / p.page_size];
+                if (pg < 0 || pg >= p.num_pages) {
+                    set_error(p.err, kErrBounds, kDetPage);
+                    pg = -1;
+                }
+            }
+            dst[sb] = pg;
+        }
+    }
+    __syncwarp();
+}
+
 // Both tiles of a work item into one stage, one barrier: the K tile only
 // adds its bytes, the V tile adds its bytes and arrives (once per phase).
 template <int D, int BLK, bool FP8>
 __device__ __forceinline__ void issue_item_loads(const KParams& p, const AttnMaps& maps,
                                                  const SeqInfo& s, int b, int hk, int item,
-                                                 uint32_t k_s, uint32_t v_s, uint64_t* full) {
-    issue_tile_load<D, BLK, FP8>(p, &maps.k, &maps.kb, s, b, hk, item, k_s, full, false);
-    issue_tile_load<D, BLK, FP8>(p, &maps.v, &maps.vb, s, b, hk, item, v_s, full, true);
+                                                 const int* pages, uint32_t k_s, uint32_t v_s,
+                                                 uint64_t* full) {
+    issue_tile_load<D, BLK, FP8>(p, &maps.k, &maps.kb, s, b, hk, item, pages, k_s, full, false);
+    issue_tile_load<D, BLK, FP8>(p, &maps.v, &maps.vb, s, b, hk, item, pages, v_s, full, true);
 }
 
 // Zeroes rows [nvalid, BLK) of a V tile (NCH chunks of BLK x 128 bytes) with

@@ -44,12 +44,14 @@ struct PairCfg {
     static constexpr int Q_BYTES = 128 * D * ELT;   // one tile
     static constexpr int KV_BYTES = BLK * D * ELT;
     static constexpr int P_COLS = BLK * ELT / 4;    // 32-bit TMEM columns of one P row
+    static constexpr int S = 2;  // ring depth of K and of V
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = 2 * Q_BYTES;
-    static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
+    static constexpr int OFF_V = OFF_K + S * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + S * KV_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + 256;
-    static constexpr int OFF_ITEMS = OFF_MISC + 64;
+    static constexpr int OFF_RING = OFF_MISC + 64;  // page ids of upcoming items
+    static constexpr int OFF_ITEMS = OFF_RING + kPageRing * kMaxBoxes * 4;
     static_assert(P_COLS % 32 == 0, "P row must be whole 32-column TMEM stores");
     // pairs (of every 4) whose exp2 runs on the FMA pipe: the fp8 MMA is twice
     // as fast, so more of the exp2 work moves off the MUFU unit there
@@ -127,8 +129,12 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     if (warp >= 8) {
       regs_decrease<56>();
-      if (warp == 8 && lane == 0) {
+      if (warp == 8) {
         // ---------------------------------------------------------- producer ---
+        // the whole warp resolves page ids 32 items at a time; lane 0 waits
+        // and issues every copy
+        int* pring = reinterpret_cast<int*>(smem + C::OFF_RING);
+        if (lane == 0) {
             prefetch_tmap(&maps.q);
             prefetch_tmap(&maps.k);
             prefetch_tmap(&maps.v);
@@ -137,44 +143,53 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 for (int c = 0; c < C::NCH; ++c)
                     tma_load_3d(q_s + x * C::Q_BYTES + c * (128 * 128), &maps.q, &bars[PB_Q_FULL],
                                 c * C::CH, hk * G, s.q0 + t_begin + x * TOK);
-            // K runs one item ahead of V: iteration n loads K(n), then V(n-1)
-            int k_issued = 0, v_issued = 0;
-            bool ok = true;
-            for (int n = 0; ok && n <= n_items; ++n) {
+        }
+        // K runs one item ahead of V: iteration n loads K(n), then V(n-1)
+        int k_issued = 0, v_issued = 0;
+        bool ok = true;
+        for (int n = 0; n <= n_items; ++n) {
+            if (n % 32 == 0 && n < n_items) fill_page_ring<BLK>(p, s, b, items, n_items, n, pring);
+            if (lane == 0) {
                 if (n < n_items) {
-                    const int st = n & 1;
-                    if (n >= 2 && !mbar_wait(&bars[PB_K_EMPTY + st], ((n - 2) >> 1) & 1,
-                                             abort_flag, kWaitLimitNs)) {
+                    const int st = n % C::S;
+                    if (n >= C::S && !mbar_wait(&bars[PB_K_EMPTY + st], ((n - C::S) / C::S) & 1,
+                                                abort_flag, kWaitLimitNs)) {
                         set_error(p.err, kErrTimeout, kDetWaitBase + 0);
                         ok = false;
-                        break;
+                    } else {
+                        issue_tile_load<D, BLK, FP8>(p, &maps.k, &maps.kb, s, b, hk, items[n],
+                                                     pring + (n % kPageRing) * kMaxBoxes,
+                                                     sbase + C::OFF_K + st * C::KV_BYTES,
+                                                     &bars[PB_K_FULL + st], true);
+                        ++k_issued;
                     }
-                    issue_tile_load<D, BLK, FP8>(p, &maps.k, &maps.kb, s, b, hk, items[n],
-                                                 sbase + C::OFF_K + st * C::KV_BYTES,
-                                                 &bars[PB_K_FULL + st], true);
-                    ++k_issued;
                 }
-                if (n >= 1) {
-                    const int m = n - 1, st = m & 1;
-                    if (m >= 2 && !mbar_wait(&bars[PB_V_EMPTY + st], ((m - 2) >> 1) & 1,
-                                             abort_flag, kWaitLimitNs)) {
+                if (ok && n >= 1) {
+                    const int m = n - 1, st = m % C::S;
+                    if (m >= C::S && !mbar_wait(&bars[PB_V_EMPTY + st], ((m - C::S) / C::S) & 1,
+                                                abort_flag, kWaitLimitNs)) {
                         set_error(p.err, kErrTimeout, kDetWaitBase + 0);
                         ok = false;
-                        break;
+                    } else {
+                        issue_tile_load<D, BLK, FP8>(p, &maps.v, &maps.vb, s, b, hk, items[m],
+                                                     pring + (m % kPageRing) * kMaxBoxes,
+                                                     sbase + C::OFF_V + st * C::KV_BYTES,
+                                                     &bars[PB_V_FULL + st], true);
+                        ++v_issued;
                     }
-                    issue_tile_load<D, BLK, FP8>(p, &maps.v, &maps.vb, s, b, hk, items[m],
-                                                 sbase + C::OFF_V + st * C::KV_BYTES,
-                                                 &bars[PB_V_FULL + st], true);
-                    ++v_issued;
                 }
             }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        }
+        if (lane == 0) {
             // never leave with copies in flight
             volatile int no_abort = 0;
-            for (int n = max(0, k_issued - 2); n < k_issued; ++n)
-                mbar_wait(&bars[PB_K_FULL + (n & 1)], (n >> 1) & 1, &no_abort, kWaitLimitNs);
-            for (int n = max(0, v_issued - 2); n < v_issued; ++n)
-                mbar_wait(&bars[PB_V_FULL + (n & 1)], (n >> 1) & 1, &no_abort, kWaitLimitNs);
+            for (int n = max(0, k_issued - C::S); n < k_issued; ++n)
+                mbar_wait(&bars[PB_K_FULL + n % C::S], (n / C::S) & 1, &no_abort, kWaitLimitNs);
+            for (int n = max(0, v_issued - C::S); n < v_issued; ++n)
+                mbar_wait(&bars[PB_V_FULL + n % C::S], (n / C::S) & 1, &no_abort, kWaitLimitNs);
             mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, kWaitLimitNs);
+        }
       } else if (warp == 9 && lane == 0) {
         // -------------------------------------------------------------- MMA ---
             constexpr uint32_t fmt = FP8 ? 0u : 1u;
