@@ -43,6 +43,8 @@ def parse():
                     help="3 = the 128K layer (the metric's workload); 2 = the 32K layer, a "
                          "smaller case for profiler captures; 5 = a 32K chunk on a "
                          "229376-token paged prefix (also times the block-mean cache)")
+    ap.add_argument("--group-masks", action="store_true",
+                    help="one mask per KV group (variant) instead of one per query head")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -218,7 +220,8 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
                           max_seqlen_q=max(s.lens_q), max_seqlen_k=max(s.lens_k),
                           seqlens_k=lk, cu_seqlens_k=cuk, page_table=pt,
                           page_size=k.shape[1] if inp.paged else 0, q_scale=sc[0],
-                          k_scale=sc[1], v_scale=sc[2], stream=stream.cuda_stream)
+                          k_scale=sc[1], v_scale=sc[2], stream=stream.cuda_stream,
+                          group_masks=args.group_masks)
     P = pr.params
     B = s.B
     with torch.cuda.stream(stream):
@@ -527,7 +530,8 @@ def main():
                    "layout": "paged K/V (64-token pages)" if synth.workload(args.workload).page_size
                    else "contiguous K/V",
                    "l2": "inputs (1.6 GB) larger than L2; no flush",
-                   "per_gpu": "one independent layer per GPU"},
+                   "per_gpu": "one independent layer per GPU",
+                   "masks": "per KV group (variant)" if args.group_masks else "per query head"},
         "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
                      "frac": eff / peak, "traffic": recorded_traffic(main_dt),
                      "kernel": "fp2_attn (attn_kernel)",

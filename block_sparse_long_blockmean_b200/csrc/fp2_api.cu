@@ -114,6 +114,7 @@ fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_
     kp.nw = L.nw;
     kp.fp8 = dtype == FP2_FP8_E4M3;
     kp.uses_kv = uses_kv ? 1 : 0;
+    kp.group_masks = P->group_masks ? 1 : 0;
     kp.cu_q = cu_seqlens;
     kp.cu_k = P->cu_seqlens_k ? P->cu_seqlens_k : cu_seqlens;
     kp.seqlens_k = P->seqlens_k;

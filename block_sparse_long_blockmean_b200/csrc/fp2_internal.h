@@ -17,6 +17,7 @@ struct KParams {
     int nqb_max, nkb_max, nw;
     int fp8;
     int uses_kv;               // 0: the launch never reads K/V (no key-extent check)
+    int group_masks;           // score every head with its group's mean pooled query
     const int32_t* cu_q;       // [S+1]
     const int32_t* cu_k;       // [S+1] contiguous key offsets (may alias cu_q)
     const int32_t* seqlens_k;  // [S] or nullptr

@@ -207,6 +207,29 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
         qb[c] = sum * inv * (FP8 ? p.q_scale[hk * G + c / D] : 1.f);
     }
     __syncthreads();
+    if (p.group_masks && G > 1) {
+        // group-shared masks: every head of the group is scored with the
+        // mean of the G pooled queries (so all G get the same mask)
+        float gm[(D + 255) / 256];
+#pragma unroll
+        for (int u = 0; u < (D + 255) / 256; ++u) {
+            const int c = threadIdx.x + u * 256;
+            float a = 0.f;
+            if (c < D)
+#pragma unroll
+                for (int g = 0; g < G; ++g) a += qb[g * D + c];
+            gm[u] = a / (float)G;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < (D + 255) / 256; ++u) {
+            const int c = threadIdx.x + u * 256;
+            if (c < D)
+#pragma unroll
+                for (int g = 0; g < G; ++g) qb[g * D + c] = gm[u];
+        }
+        __syncthreads();
+    }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int PER_LANE = D / 32;  // 4 (d=128) or 2 (d=64)

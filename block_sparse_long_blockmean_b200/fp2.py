@@ -56,6 +56,7 @@ class Params(ctypes.Structure):
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p),
+        ("group_masks", ctypes.c_int),
     ]
 
 
@@ -277,7 +278,8 @@ class Problem:
 def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, dtype: int,
                  max_seqlen_q: int, max_seqlen_k: int, seqlens_k=None, cu_seqlens_k=None,
                  page_table=None, page_size: int = 0, q_scale=None, k_scale=None,
-                 v_scale=None, out=None, stream=None, workspace=None) -> Problem:
+                 v_scale=None, out=None, stream=None, workspace=None,
+                 group_masks: bool = False) -> Problem:
     """Builds fp2_params for device tensors and allocates the workspace and
     the bf16 output with torch (allocation only)."""
     import torch
@@ -297,6 +299,7 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
     P.seqlens_k = _ptr(seqlens_k)
     P.cu_seqlens_k = _ptr(cu_seqlens_k)
     P.q_scale, P.k_scale, P.v_scale = _ptr(q_scale), _ptr(k_scale), _ptr(v_scale)
+    P.group_masks = 1 if group_masks else 0
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
     P.stream = stream

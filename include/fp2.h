@@ -95,6 +95,10 @@ typedef struct fp2_params {
     void* workspace;           /* device, fp2_workspace_size() bytes, 256-byte aligned */
     size_t workspace_bytes;
     void* stream;              /* cudaStream_t */
+    int group_masks;           /* 0 (default): one mask per query head.  1: one mask per KV
+                                  group (a variant): fp2_score scores every head of a group
+                                  with the group-mean pooled query, so all G heads keep the
+                                  same blocks and PackGQA walks no union of differing lists */
 } fp2_params;
 
 /* Offsets (bytes from params->workspace) of the intermediates, for callers

@@ -174,11 +174,21 @@ class SeqResult:
         self.out, self.rows, self.heads = out, rows, heads
 
 
+def group_pool(qbar, Hkv: int):
+    """Group-shared masks (a variant): the pooled query of a KV group is the
+    mean of its G heads' pooled queries, [Hkv, nqb, d]."""
+    Hq, nqb, d = qbar.shape
+    return np.asarray(qbar).reshape(Hkv, Hq // Hkv, nqb, d).mean(axis=1)
+
+
 def prefill_seq(Q, K, V, B: int, tau: float, rows=None, heads=None, keep=None,
-                mutant: int = 0) -> SeqResult:
+                group_masks: bool = False, mutant: int = 0) -> SeqResult:
     """All steps for one sequence: block means, pooled scores, threshold mask
     (unless ``keep`` is given), then the corrected sparse attention on the
-    requested (row, head) pairs (all of them by default)."""
+    requested (row, head) pairs (all of them by default).  With
+    ``group_masks`` every head of a KV group takes the group's mask, scored
+    with the group-mean pooled query; ``S`` then holds the group score in
+    each head's row."""
     Lq, Hq, _ = np.shape(Q)
     Lk = np.shape(K)[0]
     P = Lk - Lq
@@ -186,7 +196,12 @@ def prefill_seq(Q, K, V, B: int, tau: float, rows=None, heads=None, keep=None,
         raise ValueError("prefix length must be a multiple of the block size")
     kbar, vbar, cnt = blockmean(K, V, B, mutant)
     qbar = pool_q(Q, B, mutant)
-    S = score(qbar, kbar, P // B, mutant)
+    if group_masks:
+        Hkv = kbar.shape[0]
+        Sg = score(group_pool(qbar, Hkv), kbar, P // B, mutant)
+        S = np.repeat(Sg, Hq // Hkv, axis=0)
+    else:
+        S = score(qbar, kbar, P // B, mutant)
     if keep is None:
         keep = mask(S, P // B, tau, mutant)
     if rows is None:

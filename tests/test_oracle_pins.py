@@ -273,3 +273,43 @@ def test_pins_pass_on_the_oracle():
 @pytest.mark.parametrize("mutant", [1, 2, 3, 4])
 def test_pins_catch_mutant(mutant):
     assert not _pins_pass(mutant)
+
+
+# --------------------------------------------------------------------------
+# group-shared masks (a variant: one mask per KV group, scored with the
+# group-mean pooled query)
+# --------------------------------------------------------------------------
+
+def test_group_masks_equal_head_masks_when_heads_agree():
+    """If the G query heads of a group carry identical queries, the group
+    mean is each head's pooled query: group masks = per-head masks, and the
+    outputs agree."""
+    rng = np.random.default_rng(12)
+    Lq, Lk, Hq, Hkv, d, B = 70, 102, 4, 2, 8, 8
+    Q, K, V = rand_seq(rng, Lq, Lk, Hq, Hkv, d, scale=1.5)
+    Q[:, 1] = Q[:, 0]
+    Q[:, 3] = Q[:, 2]
+    a = O.prefill_seq(Q, K, V, B, 0.6)
+    g = O.prefill_seq(Q, K, V, B, 0.6, group_masks=True)
+    assert (a.keep == g.keep).all()
+    np.testing.assert_allclose(a.out, g.out, atol=1e-13)
+
+
+def test_group_masks_use_the_mean_query():
+    """Hand-made: one KV head, two query heads, d = 1, B = 2, 6 tokens.
+    Queries: head 0 = +2, head 1 = -1 (group mean +0.5).  Keys: block0 = [1, 1],
+    block1 = [-3, -3], block2 = [0.2, 0.2].  Query block 2 scores: per head 0:
+    (2, -6, 0.4), per head 1: (-1, 3, -0.2), group: (0.5, -1.5, 0.1).  With
+    tau = 1 the per-head masks are head 0: {0, 2}, head 1: {1 (the max), 0 and
+    2 forced} -> [1,1,1]; the group mask keeps {0, 2} (-1.5 < 0.5 - 1) for both
+    heads."""
+    K = np.array([1, 1, -3, -3, 0.2, 0.2], dtype=np.float64).reshape(6, 1, 1)
+    V = np.arange(6, dtype=np.float64).reshape(6, 1, 1)
+    Q = np.zeros((6, 2, 1))
+    Q[:, 0] = 2.0
+    Q[:, 1] = -1.0
+    a = O.prefill_seq(Q, K, V, 2, 1.0)
+    g = O.prefill_seq(Q, K, V, 2, 1.0, group_masks=True)
+    assert a.keep[0, 2].tolist() == [1, 0, 1] and a.keep[1, 2].tolist() == [1, 1, 1]
+    assert g.keep[0, 2].tolist() == [1, 0, 1] and g.keep[1, 2].tolist() == [1, 0, 1]
+    np.testing.assert_allclose(g.S[:, 2], [[0.5, -1.5, 0.1]] * 2, atol=1e-15)
