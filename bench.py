@@ -43,6 +43,8 @@ def parse():
                     help="3 = the 128K layer (the metric's workload); 2 = the 32K layer, a "
                          "smaller case for profiler captures; 5 = a 32K chunk on a "
                          "229376-token paged prefix (also times the block-mean cache)")
+    ap.add_argument("--out-fp8", action="store_true",
+                    help="e4m3 output (fp8 runs; default scale: the KV head's v_scale)")
     ap.add_argument("--group-masks", action="store_true",
                     help="one mask per KV group (variant) instead of one per query head")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -221,7 +223,9 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
                           seqlens_k=lk, cu_seqlens_k=cuk, page_table=pt,
                           page_size=k.shape[1] if inp.paged else 0, q_scale=sc[0],
                           k_scale=sc[1], v_scale=sc[2], stream=stream.cuda_stream,
-                          group_masks=args.group_masks)
+                          group_masks=args.group_masks,
+                          out_dtype=fp2.FP2_FP8_E4M3 if (args.out_fp8 and dtype_name == "fp8")
+                          else fp2.FP2_BF16)
     P = pr.params
     B = s.B
     with torch.cuda.stream(stream):
@@ -298,7 +302,7 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
             hq = inp.q.pin_memory()
             hk = inp.k.pin_memory()
             hv = inp.v.pin_memory()
-            hout = torch.empty(pr.out.shape, dtype=torch.bfloat16).pin_memory()
+            hout = torch.empty(pr.out.shape, dtype=pr.out.dtype).pin_memory()
             nsteps = max(2, min(args.steps, 5))
             for it in range(nsteps + 1):
                 if it == 1:
@@ -531,7 +535,8 @@ def main():
                    else "contiguous K/V",
                    "l2": "inputs (1.6 GB) larger than L2; no flush",
                    "per_gpu": "one independent layer per GPU",
-                   "masks": "per KV group (variant)" if args.group_masks else "per query head"},
+                   "masks": "per KV group (variant)" if args.group_masks else "per query head",
+                   "output": "e4m3 for the fp8 run" if args.out_fp8 else "bf16"},
         "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
                      "frac": eff / peak, "traffic": recorded_traffic(main_dt),
                      "kernel": "fp2_attn (attn_kernel)",

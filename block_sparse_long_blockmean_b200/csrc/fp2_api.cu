@@ -44,6 +44,9 @@ fp2_status check_kv(const fp2_params* P, int block, const int32_t* page_table) {
 }
 
 fp2_status check_dtype(const fp2_params* P, int block, fp2_dtype dtype) {
+    if (P->out_dtype != FP2_BF16 && P->out_dtype != FP2_FP8_E4M3) return FP2_ERR_INVALID_ARG;
+    if (P->out_dtype == FP2_FP8_E4M3 && dtype == FP2_BF16 && !P->out_scale)
+        return FP2_ERR_INVALID_ARG;
     if (dtype == FP2_BF16) return FP2_OK;
     if (dtype != FP2_FP8_E4M3) return FP2_ERR_INVALID_ARG;
     if (P->head_dim != 128 || block != 128) return FP2_ERR_UNSUPPORTED;
@@ -115,6 +118,8 @@ fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_
     kp.fp8 = dtype == FP2_FP8_E4M3;
     kp.uses_kv = uses_kv ? 1 : 0;
     kp.group_masks = P->group_masks ? 1 : 0;
+    kp.out_fp8 = P->out_dtype == FP2_FP8_E4M3;
+    kp.out_scale = P->out_scale;
     kp.cu_q = cu_seqlens;
     kp.cu_k = P->cu_seqlens_k ? P->cu_seqlens_k : cu_seqlens;
     kp.seqlens_k = P->seqlens_k;

@@ -247,6 +247,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         const bool row_ok = t < s.Lq;
         const int ppos = s.P + t;                // absolute position
         const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
+        const uint32_t o_addr = tmem + lane_off + 256;
         const uint32_t* hb = sbits + g * nw_c;
         float sl2 = rsqrtf((float)D) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e)
         if constexpr (FP8) sl2 *= p.q_scale[h] * p.k_scale[hk];
@@ -387,12 +388,37 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                                                     abort_flag, kWaitLimitNs))) {
             tc_fence_after();
             float inv = l > 0.f ? 1.f / l : 0.f;
+            if (p.out_fp8) {
+                // e4m3 output in units of out_scale[h] (default: the KV head's
+                // v_scale, the units O has before dequantisation)
+                float vs = FP8 ? p.v_scale[hk] : 1.f;
+                if (p.out_scale) inv *= vs / p.out_scale[h];
+                else if (!FP8) inv = 0.f;  // rejected on the host; never reached
+                uint8_t* orow8 = reinterpret_cast<uint8_t*>(out) + ((size_t)(s.q0 + t) * p.Hq + h) * D;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + c * 32, o);
+                    tmem_wait_ld();
+                    if (row_ok) {
+                        uint32_t wd[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            wd[e] = pack_e4m3x4(__uint_as_float(o[4 * e]) * inv,
+                                                __uint_as_float(o[4 * e + 1]) * inv,
+                                                __uint_as_float(o[4 * e + 2]) * inv,
+                                                __uint_as_float(o[4 * e + 3]) * inv);
+                        *reinterpret_cast<uint4*>(orow8 + c * 32) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                        *reinterpret_cast<uint4*>(orow8 + c * 32 + 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+                    }
+                }
+            } else {
             if constexpr (FP8) inv *= p.v_scale[hk];
             __nv_bfloat16* orow = out + ((size_t)(s.q0 + t) * p.Hq + h) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
-                tmem_ld32(tmem + lane_off + 256 + c * 32, o);
+                tmem_ld32(o_addr + c * 32, o);
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
@@ -409,6 +435,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                             make_uint4(wd[0], wd[1], wd[2], wd[3]);
                     }
                 }
+            }
             }
         } else if (ok) {
             set_error(p.err, kErrTimeout, kDetWaitBase + 6);

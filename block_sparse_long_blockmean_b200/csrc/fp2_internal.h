@@ -18,6 +18,8 @@ struct KParams {
     int fp8;
     int uses_kv;               // 0: the launch never reads K/V (no key-extent check)
     int group_masks;           // score every head with its group's mean pooled query
+    int out_fp8;               // e4m3 output (O / out_scale), else bf16
+    const float* out_scale;    // [Hq] or nullptr (FP8 inputs: v_scale of the KV head)
     const int32_t* cu_q;       // [S+1]
     const int32_t* cu_k;       // [S+1] contiguous key offsets (may alias cu_q)
     const int32_t* seqlens_k;  // [S] or nullptr

@@ -57,6 +57,8 @@ class Params(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p),
         ("group_masks", ctypes.c_int),
+        ("out_dtype", ctypes.c_int),
+        ("out_scale", ctypes.c_void_p),
     ]
 
 
@@ -279,7 +281,8 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
                  max_seqlen_q: int, max_seqlen_k: int, seqlens_k=None, cu_seqlens_k=None,
                  page_table=None, page_size: int = 0, q_scale=None, k_scale=None,
                  v_scale=None, out=None, stream=None, workspace=None,
-                 group_masks: bool = False) -> Problem:
+                 group_masks: bool = False, out_dtype: int = FP2_BF16,
+                 out_scale=None) -> Problem:
     """Builds fp2_params for device tensors and allocates the workspace and
     the bf16 output with torch (allocation only)."""
     import torch
@@ -300,6 +303,8 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
     P.cu_seqlens_k = _ptr(cu_seqlens_k)
     P.q_scale, P.k_scale, P.v_scale = _ptr(q_scale), _ptr(k_scale), _ptr(v_scale)
     P.group_masks = 1 if group_masks else 0
+    P.out_dtype = out_dtype
+    P.out_scale = _ptr(out_scale)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
     P.stream = stream
@@ -312,6 +317,7 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
     P.workspace_bytes = workspace.numel()
     workspace_init(P)
     if out is None:
-        out = torch.empty((q.shape[0], Hq, d), dtype=torch.bfloat16, device=dev)
-    keep = (seqlens_k, cu_seqlens_k, q_scale, k_scale, v_scale)
+        odt = torch.float8_e4m3fn if out_dtype == FP2_FP8_E4M3 else torch.bfloat16
+        out = torch.empty((q.shape[0], Hq, d), dtype=odt, device=dev)
+    keep = (seqlens_k, cu_seqlens_k, q_scale, k_scale, v_scale, out_scale)
     return Problem(q, k, v, page_table, cu_seqlens, out, block, dtype, P, workspace, keep)

@@ -99,6 +99,11 @@ typedef struct fp2_params {
                                   group (a variant): fp2_score scores every head of a group
                                   with the group-mean pooled query, so all G heads keep the
                                   same blocks and PackGQA walks no union of differing lists */
+    int out_dtype;             /* FP2_BF16 (default): out is bf16.  FP2_FP8_E4M3: out is e4m3
+                                  [total_q, Hq, d] holding O / out_scale[h], saturating */
+    const float* out_scale;    /* device [Hq], e4m3 output only.  NULL with FP8 inputs: the
+                                  KV head's v_scale (|O| <= max|V|, so it never saturates);
+                                  required with BF16 inputs */
 } fp2_params;
 
 /* Offsets (bytes from params->workspace) of the intermediates, for callers

@@ -148,6 +148,14 @@ def test_calls_reject_bad_arguments_before_any_cuda_work(lib):
     assert lib.fp2_prefill(fake, fake, fake, fake, fake, 1.0, 128, 0, fake,
                            ctypes.byref(P)) == fp2.FP2_ERR_INVALID_ARG
     assert lib.fp2_mask(fake, float("nan"), 128, ctypes.byref(P)) == fp2.FP2_ERR_INVALID_ARG
+    # e4m3 output from bf16 inputs needs an explicit out_scale; unknown out dtype
+    P.page_size, P.max_pages_per_seq = 64, 4
+    P.out_dtype = fp2.FP2_FP8_E4M3
+    assert lib.fp2_prefill(fake, fake, fake, None, fake, 1.0, 128, 0, fake,
+                           ctypes.byref(P)) == fp2.FP2_ERR_INVALID_ARG
+    P.out_dtype = 5
+    assert lib.fp2_prefill(fake, fake, fake, None, fake, 1.0, 128, 0, fake,
+                           ctypes.byref(P)) == fp2.FP2_ERR_INVALID_ARG
 
 
 def test_status_strings_and_version(lib):
