@@ -36,7 +36,14 @@
  *
  * Layouts (all fp64, row-major, one sequence per call):
  *   Q [Lq][Hq][d], K and V [Lk][Hkv][d]; query t sits at absolute position
- *   P + t with P = Lk - Lq (a resident prefix), P % B == 0.
+ *   P + t with P = Lk - Lq (a resident prefix, any length >= 0).  Blocks are
+ *   cut at absolute positions, for queries as for keys: query block i of the
+ *   call is absolute block P/B + i (integer division) and holds the call's
+ *   rows that fall in [(P/B + i)B, (P/B + i + 1)B).  When P is not a multiple
+ *   of B the first query block is partial (READING: the pages' "mixed
+ *   prefill + decode chunk" puts rows at arbitrary positions; a decode row is
+ *   a call with Lq = 1), and its pooled query is the mean of the rows it
+ *   holds.  nqb = ceil((P mod B + Lq) / B).
  *   kbar, vbar [Hkv][nkb][d]; cnt [nkb]; qbar [Hq][nqb][d];
  *   S [Hq][nqb][nkb] (entries with j > i_abs are left untouched);
  *   keep [Hq][nqb][nkb] bytes, 1 = kept, 0 = dropped or non-causal.
@@ -48,7 +55,9 @@
  * a plausible slip): 1 drops the ln(n_j) term, 2 flips the inequality of the
  * threshold to strict and forgets the forced diagonal, 3 adds the correction
  * term's weight to the numerator only, 4 uses the mean of the first row of a
- * block's keys instead of the mean of the block.
+ * block's keys instead of the mean of the block, 5 picks a row's mask by its
+ * offset in the call (t / B) instead of its absolute block, 6 pools the
+ * query blocks as if the prefix were a multiple of B.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -88,12 +97,18 @@ void oracle_blockmean(const double* K, const double* V, int Lk, int Hkv, int d, 
     }
 }
 
-/* ---- step: pooled query blocks ([ABS] instantaneous pattern discovery) --- */
-void oracle_pool_q(const double* Q, int Lq, int Hq, int d, int B, double* qbar)
+/* ---- step: pooled query blocks ([ABS] instantaneous pattern discovery) ---
+ * off = P mod B, the offset of the call's first row inside its block. */
+void oracle_pool_q(const double* Q, int Lq, int Hq, int d, int B, int off, double* qbar)
 {
-    int nqb = ceil_div(Lq, B);
+    int nqb = ceil_div(off + Lq, B);
+#if FP2_ORACLE_MUTANT == 6
+    off = 0;
+#endif
     for (int i = 0; i < nqb; ++i) {
-        int t0 = i * B, t1 = (i + 1) * B < Lq ? (i + 1) * B : Lq;
+        int t0 = i * B - off, t1 = (i + 1) * B - off;
+        if (t0 < 0) t0 = 0;
+        if (t1 > Lq) t1 = Lq;
         for (int h = 0; h < Hq; ++h)
             for (int c = 0; c < d; ++c) {
                 double s = 0.0;
@@ -162,14 +177,18 @@ void oracle_attn_rows(const double* Q, const double* K, const double* V,
 {
     int G = Hq / Hkv;
     int P = Lk - Lq;
-    int nqb = ceil_div(Lq, B), nkb = ceil_div(Lk, B);
+    int nqb = ceil_div(P % B + Lq, B), nkb = ceil_div(Lk, B);
     double scale = 1.0 / sqrt((double)d);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < nrows; ++r) {
         int t = rows[r], h = heads[r], hk = h / G;
         int p = P + t;
-        int i = t / B;              /* local query block */
         int iabs = p / B;           /* absolute query block */
+#if FP2_ORACLE_MUTANT == 5
+        int i = t / B;
+#else
+        int i = iabs - P / B;       /* query block of the call */
+#endif
         const double* q = Q + ((size_t)t * Hq + h) * d;
         const unsigned char* kr = keep + ((size_t)h * nqb + i) * nkb;
         /* logits and values: at most Lk tokens + nkb pseudo-tokens */

@@ -56,7 +56,7 @@ def _lib(mutant: int = 0) -> ctypes.CDLL:
             lib.oracle_blockmean.argtypes = [_D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, _D, _D, _I]
             lib.oracle_pool_q.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                          ctypes.c_int, _D]
+                                          ctypes.c_int, ctypes.c_int, _D]
             lib.oracle_score.argtypes = [_D, _D] + [ctypes.c_int] * 6 + [_D]
             lib.oracle_mask.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_double, _U8]
@@ -93,13 +93,14 @@ def blockmean(K, V, B: int, mutant: int = 0):
     return kbar, vbar, cnt
 
 
-def pool_q(Q, B: int, mutant: int = 0):
-    """Pooled query blocks ``qbar [Hq, nqb, d]`` (mean over the valid rows)."""
+def pool_q(Q, B: int, off: int = 0, mutant: int = 0):
+    """Pooled query blocks ``qbar [Hq, nqb, d]`` (mean over the valid rows);
+    ``off`` = prefix mod B, the offset of row 0 inside its block."""
     Q = _f64(Q)
     Lq, Hq, d = Q.shape
-    nqb = -(-Lq // B)
+    nqb = -(-(off + Lq) // B)
     qbar = np.zeros((Hq, nqb, d))
-    _lib(mutant).oracle_pool_q(_p(Q, _D), Lq, Hq, d, B, _p(qbar, _D))
+    _lib(mutant).oracle_pool_q(_p(Q, _D), Lq, Hq, d, B, off, _p(qbar, _D))
     return qbar
 
 
@@ -192,10 +193,10 @@ def prefill_seq(Q, K, V, B: int, tau: float, rows=None, heads=None, keep=None,
     Lq, Hq, _ = np.shape(Q)
     Lk = np.shape(K)[0]
     P = Lk - Lq
-    if P % B != 0:
-        raise ValueError("prefix length must be a multiple of the block size")
+    if P < 0:
+        raise ValueError("more queries than keys")
     kbar, vbar, cnt = blockmean(K, V, B, mutant)
-    qbar = pool_q(Q, B, mutant)
+    qbar = pool_q(Q, B, P % B, mutant)
     if group_masks:
         Hkv = kbar.shape[0]
         Sg = score(group_pool(qbar, Hkv), kbar, P // B, mutant)
@@ -261,19 +262,24 @@ def tau_for_drop(S_list, prefix_blocks_list, target: float, guard: float = 0.0):
 
 
 def attn_query_block(Qblk, K, V, kbar, vbar, cnt, keep_i, B: int, iabs: int, heads=None,
-                     mutant: int = 0):
+                     p0: int | None = None, mutant: int = 0):
     """Corrected attention of ONE query block at absolute block index ``iabs``.
 
-    ``Qblk`` [n, Hq, d] holds the block's rows, ``keep_i`` [Hq, >= iabs+1] its
-    mask row.  Calls ``attn_rows`` on the causal window: keys ``[0, iabs*B+n)``
-    (later keys never reach these rows) with the block as the whole query
-    side, so that prefix = iabs*B puts every row at its true position.  No
-    arithmetic of its own; it lets a long sequence be checked block by block
-    without an fp64 copy of all of Q.  Returns [n * len(heads), d] ordered
-    (row, head)."""
+    ``Qblk`` [n, Hq, d] holds the block's rows, the first at absolute position
+    ``p0`` (default ``iabs*B``; later for the partial first block of a call
+    whose prefix is not a multiple of B), ``keep_i`` [Hq, >= iabs+1] its mask
+    row.  Calls ``attn_rows`` on the causal window: keys ``[0, p0+n)`` (later
+    keys never reach these rows) with the block as the whole query side, so
+    that prefix = p0 puts every row at its true position.  No arithmetic of
+    its own; it lets a long sequence be checked block by block without an
+    fp64 copy of all of Q.  Returns [n * len(heads), d] ordered (row, head)."""
     Qblk = _f64(Qblk)
     n, Hq, d = Qblk.shape
-    Lk = iabs * B + n
+    if p0 is None:
+        p0 = iabs * B
+    if p0 // B != iabs or (p0 + n - 1) // B != iabs:
+        raise ValueError("the rows must lie in block iabs")
+    Lk = p0 + n
     nkb = iabs + 1
     if heads is None:
         heads = np.arange(Hq, dtype=np.int32)

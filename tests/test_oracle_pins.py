@@ -13,7 +13,11 @@ exactly that.
 * uniform attention (q = 0): output = mean of V over the causal prefix for
   every tau (closed form);
 * a hand-worked 3-block case with one dropped block;
-* block means / pooled queries / scores == numpy mean and einsum;
+* block means / pooled queries / scores == numpy mean and einsum, with the
+  query blocks cut at absolute positions when the prefix is not a multiple
+  of the block (decode rows, arbitrary chunk boundaries);
+* a decode row given the full prefill's mask equals the full prefill's last
+  row;
 * threshold: hand-made score rows with obvious kept sets (max-based dynamic
   thresholding of the FlashPrefill V2 abstract, plus the forced first and
   diagonal blocks);
@@ -55,6 +59,10 @@ SHAPES = [  # Lq, Lk, Hq, Hkv, d, B
     (29, 61, 4, 1, 8, 8),     # prefix of 32 (4 blocks of 8), ragged tail
     (50, 50, 8, 8, 4, 4),
     (9, 9, 1, 1, 3, 16),      # one partial block
+    (1, 61, 4, 1, 8, 8),      # a decode row: one query at position 60 (block 7, offset 4)
+    (13, 50, 2, 1, 8, 8),     # prefix 37: the first query block holds 3 rows
+    (5, 23, 4, 2, 4, 16),     # prefix 18: the whole call inside one block
+    (40, 47, 4, 2, 8, 8),     # prefix 7: first query block of 1 row, ragged tail
 ]
 
 
@@ -189,6 +197,42 @@ def test_blockmean_pool_score_match_numpy():
         assert np.isnan(S[:, i, iabs + 1:]).all()
 
 
+@pytest.mark.parametrize("Lq,P,B", [(1, 60, 8), (13, 37, 8), (5, 18, 16), (40, 7, 8),
+                                     (24, 16, 8)])
+def test_pool_q_cuts_blocks_at_absolute_positions(Lq, P, B):
+    """The call's query blocks follow the absolute blocks: row t belongs to
+    block (P + t) // B - P // B, and each pooled query is the numpy mean of
+    exactly those rows."""
+    rng = np.random.default_rng(13)
+    Q = rng.standard_normal((Lq, 3, 5))
+    qbar = O.pool_q(Q, B, P % B)
+    lab = (P + np.arange(Lq)) // B - P // B
+    assert qbar.shape[1] == lab[-1] + 1
+    for i in range(qbar.shape[1]):
+        np.testing.assert_allclose(qbar[:, i], Q[lab == i].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_decode_row_keeps_and_corrects_like_a_prefill_row():
+    """A decode row (Lq = 1) at position p is the last row of the same
+    sequence's full prefill when the masks agree: with the mask of the full
+    prefill's last query block given explicitly, the two outputs coincide
+    (same kept tokens, same pseudo-tokens)."""
+    rng = np.random.default_rng(14)
+    L, Hq, Hkv, d, B = 77, 4, 2, 8, 8
+    Q, K, V = rand_seq(rng, L, L, Hq, Hkv, d, scale=1.5)
+    full = O.prefill_seq(Q, K, V, B, 0.4)
+    assert full.keep.sum() < np.isfinite(full.S).sum()  # something is dropped
+    keep_last = full.keep[:, -1:, :]
+    one = O.prefill_seq(Q[-1:], K, V, B, 0.4, keep=keep_last)
+    want = full.out.reshape(L, Hq, d)[-1]
+    np.testing.assert_allclose(one.out.reshape(Hq, d), want, rtol=0, atol=1e-13)
+    # and the decode row's own mask is scored with its own query, not the block mean
+    own = O.prefill_seq(Q[-1:], K, V, B, 0.4)
+    G = Hq // Hkv
+    qs = np.einsum("hd,hjd->hj", Q[-1], np.repeat(own.kbar, G, axis=0)) / math.sqrt(d)
+    np.testing.assert_allclose(own.S[:, 0, :], qs, rtol=0, atol=1e-13)
+
+
 def test_mask_hand_made_rows():
     # one head, one query block at absolute index 4 (prefix of 4 blocks)
     S = np.array([[[5.0, 1.0, 4.5, 0.0, 2.0, np.nan]]])
@@ -263,6 +307,13 @@ def _pins_pass(mutant: int) -> bool:
     Qr, Kr, Vr = rand_seq(rng, 45, 77, 4, 2, 8)
     kbar, _, _ = O.blockmean(Kr, Vr, 16, mutant=mutant)
     ok &= np.abs(kbar[:, 1] - Kr[16:32].mean(axis=0)).max() < 1e-14
+    # a prefix that is not a multiple of the block: constant blocks, only the
+    # forced blocks kept, still exact; pooled queries follow absolute blocks
+    Qu, Ku, Vu = constant_block_seq(rng, 29, 63, 4, 1, 8, 8)
+    ru = O.prefill_seq(Qu, Ku, Vu, 8, -1e9, mutant=mutant)
+    ok &= np.abs(ru.out - O.dense_rows(Qu, Ku, Vu, ru.rows, ru.heads)).max() < 1e-12
+    qb = O.pool_q(Qu, 8, 34 % 8, mutant=mutant)
+    ok &= qb.shape[1] == 4 and np.abs(qb[:, 0] - Qu[:6].mean(axis=0)).max() < 1e-14
     return bool(ok)
 
 
@@ -270,7 +321,7 @@ def test_pins_pass_on_the_oracle():
     assert _pins_pass(0)
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6])
 def test_pins_catch_mutant(mutant):
     assert not _pins_pass(mutant)
 
