@@ -59,8 +59,12 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 void layout_of(const fp2_params* P, int block, fp2_workspace_layout* L) {
     const size_t S = (size_t)P->num_seqs, Hq = (size_t)P->num_q_heads,
                  Hkv = (size_t)P->num_kv_heads, d = (size_t)P->head_dim;
-    const int nqb = (P->max_seqlen_q + block - 1) / block;
+    // A call's query blocks follow the absolute blocks, so a sequence whose
+    // prefix is not a multiple of the block spans up to one block more than
+    // its queries alone would: ceil((P % B + Lq) / B) <= (Lq + 2B - 2) / B,
+    // and never more than its keys' blocks.
     const int nkb = (P->max_seqlen_k + block - 1) / block;
+    const int nqb = std::min((P->max_seqlen_q + 2 * block - 2) / block, nkb);
     const int nw = (nkb + 31) / 32;
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -341,11 +345,10 @@ fp2_status fp2_calibrate_tau(const int32_t* cu_seqlens, int block, float target_
     std::vector<float> slab((size_t)kp.nqb_max * kp.nkb_max);
     for (int b = 0; b < S; ++b) {
         const int Lq = cu[b + 1] - cu[b];
-        if (Lq < 0 || Lq > kp.max_seqlen_q || lk[b] < Lq || lk[b] > kp.max_seqlen_k ||
-            (lk[b] - Lq) % block != 0)
+        if (Lq < 0 || Lq > kp.max_seqlen_q || lk[b] < Lq || lk[b] > kp.max_seqlen_k)
             return FP2_ERR_INVALID_ARG;
         const int pb = (lk[b] - Lq) / block;
-        const int nqb = (Lq + block - 1) / block;
+        const int nqb = Lq > 0 ? ((lk[b] - Lq) % block + Lq + block - 1) / block : 0;
         for (int h = 0; h < kp.Hq; ++h) {
             const size_t off = ((size_t)b * kp.Hq + h) * kp.nqb_max * kp.nkb_max;
             if (cudaMemcpy(slab.data(), kp.scores + off, (size_t)nqb * kp.nkb_max * 4,

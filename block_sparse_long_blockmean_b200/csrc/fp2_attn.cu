@@ -95,9 +95,10 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
-    const int t_begin = i * BLK + tq * TOK;
-    if (t_begin >= s.Lq) return;  // whole CTA: nothing to do
-    const int iabs = s.P / BLK + i;
+    // the tile's first query (negative inside a partial first query block)
+    const int t_begin = i * BLK - s.off + tq * TOK;
+    if (i >= s.nqb || t_begin >= s.Lq || t_begin + TOK <= 0) return;  // no rows here
+    const int iabs = s.pb + i;
     const int nw_c = (iabs + 32) / 32;  // words covering blocks 0..iabs
 
     // ---------------------------------------------------------- set-up ---
@@ -244,7 +245,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         const int tl = r / G;
         const int t = t_begin + tl;              // query index in the sequence
         const int h = hk * G + g;
-        const bool row_ok = t < s.Lq;
+        const bool row_ok = t >= 0 && t < s.Lq;
         const int ppos = s.P + t;                // absolute position
         const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
         const uint32_t o_addr = tmem + lane_off + 256;

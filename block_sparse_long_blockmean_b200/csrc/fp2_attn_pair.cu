@@ -99,9 +99,10 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
-    const int t_begin = i * BLK + pr * 2 * TOK;
-    if (t_begin >= s.Lq) return;
-    const int iabs = s.P / BLK + i;
+    // the pair's first query (negative inside a partial first query block)
+    const int t_begin = i * BLK - s.off + pr * 2 * TOK;
+    if (i >= s.nqb || t_begin >= s.Lq || t_begin + 2 * TOK <= 0) return;  // no rows here
+    const int iabs = s.pb + i;
     const int nw_c = (iabs + 32) / 32;
 
     if (threadIdx.x == 0) {
@@ -268,7 +269,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         const int g = r % G;
         const int t = t_begin + X * TOK + r / G;  // query index in the sequence
         const int h = hk * G + g;
-        const bool row_ok = t < s.Lq;
+        const bool row_ok = t >= 0 && t < s.Lq;
         const int ppos = s.P + t;
         const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + X * 128;

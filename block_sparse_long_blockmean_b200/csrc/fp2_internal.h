@@ -47,7 +47,6 @@ struct KParams {
 // Detail codes stored beside an error code.
 enum : uint32_t {
     kDetSeqLen = 1,      // Lq or Lk outside [0, max_seqlen_*] or Lk < Lq
-    kDetPrefix = 2,      // (Lk - Lq) % block != 0
     kDetPage = 3,        // page id outside [0, num_pages)
     kDetSlot = 4,        // block-mean cache slot outside [0, num_slots) or beyond max_blocks
     kDetWaitBase = 16,   // + pipeline wait site

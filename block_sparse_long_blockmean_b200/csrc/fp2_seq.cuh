@@ -12,6 +12,13 @@ struct SeqInfo {
     int k0;  // first row in contiguous K/V (0 when paged)
     int Lk;  // keys (resident prefix + new tokens)
     int P;   // prefix length Lk - Lq; query t sits at absolute position P + t
+    // Query blocks are cut at absolute positions: query block i of the call
+    // is absolute block pb + i and holds the rows t with (P + t) / B == pb + i.
+    // When P is not a multiple of B (a decode row, a chunk that ends inside a
+    // block) the first one starts `off` rows into its block and is partial.
+    int pb;   // P / B
+    int off;  // P % B
+    int nqb;  // query blocks of the call: ceil((off + Lq) / B), 0 when Lq = 0
 };
 
 // Reads sequence b's lengths and checks them against the launch's limits.
@@ -31,10 +38,9 @@ __device__ __forceinline__ bool load_seq(const KParams& p, int b, SeqInfo& s) {
         set_error(p.err, lens_ok ? kErrBounds : kErrInvalid, kDetSeqLen);
         return false;
     }
-    if (s.P % p.B != 0) {
-        set_error(p.err, kErrUnsupported, kDetPrefix);
-        return false;
-    }
+    s.pb = s.P / p.B;
+    s.off = s.P - s.pb * p.B;
+    s.nqb = s.Lq > 0 ? (s.off + s.Lq + p.B - 1) / p.B : 0;
     return true;
 }
 

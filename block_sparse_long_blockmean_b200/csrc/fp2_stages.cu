@@ -161,11 +161,11 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
     const int i = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
-    const int nqb = (s.Lq + p.B - 1) / p.B;
-    if (i >= nqb) return;
-    const int t0 = i * p.B;
-    const int n = min(p.B, s.Lq - t0);
-    const int iabs = s.P / p.B + i;
+    if (i >= s.nqb) return;
+    // rows of query block i (the first may start inside its block)
+    const int t0 = max(0, i * p.B - s.off);
+    const int n = min(s.Lq, (i + 1) * p.B - s.off) - t0;
+    const int iabs = s.pb + i;
 
     const int v = threadIdx.x % VPT, tg = threadIdx.x / VPT;
     float acc[VEC];
@@ -318,9 +318,8 @@ __global__ void __launch_bounds__(128) mask_kernel(KParams p, float tau) {
     const int b = (int)(row / ((long long)p.nqb_max * p.Hq));
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
-    const int nqb = (s.Lq + p.B - 1) / p.B;
-    if (i >= nqb) return;
-    const int iabs = s.P / p.B + i;
+    if (i >= s.nqb) return;
+    const int iabs = s.pb + i;
     const float* S = p.scores + (size_t)row * p.nkb_max;
     float m = -INFINITY;
     for (int j = lane; j <= iabs; j += 32) m = fmaxf(m, S[j]);

@@ -32,11 +32,16 @@
  *    page_table int32 [num_seqs, max_pages_per_seq] of physical page ids.
  *  - Sequence b has Lq = cu_seqlens[b+1]-cu_seqlens[b] new tokens and
  *    Lk = seqlens_k[b] (or Lq when seqlens_k is NULL) keys; query t sits at
- *    absolute position Lk - Lq + t.  Lk - Lq (the resident prefix) must be a
- *    multiple of the block size.
+ *    absolute position P + t, P = Lk - Lq (the resident prefix, any length:
+ *    a decode row is a sequence with Lq = 1).  Query blocks are cut at
+ *    absolute positions, like key blocks: query block i of sequence b is
+ *    absolute block P/B + i and holds the rows t with (P + t)/B = P/B + i, so
+ *    when P is not a multiple of B the first one is partial (explainer
+ *    section 2.3: a chunk may mix prefill and decode rows).
  *  - dtype FP2_BF16: q/k/v are bf16.  FP2_FP8_E4M3: q/k/v are e4m3 with
  *    per-head dequantisation scales (x = e4m3 * scale), params->q_scale [Hq],
- *    k_scale [Hkv], v_scale [Hkv] (fp32, device).  out is always bf16.
+ *    k_scale [Hkv], v_scale [Hkv] (fp32, device).  out is bf16 unless
+ *    params->out_dtype asks for e4m3.
  *  - Base pointers of q, k_cache, v_cache and out must be 16-byte aligned.
  *  - Supported: head_dim 64 or 128 (FP8: 128), block 64 or 128,
  *    G = Hq/Hkv in {1,2,4,8} with 128/G <= block, page_size a power of two
@@ -48,7 +53,7 @@
  *
  * Errors: argument errors are returned synchronously before any launch.
  * CUDA launch errors return FP2_ERR_CUDA.  Problems only the device can see
- * (a prefix that is not a multiple of the block, Lk < Lq, a length above
+ * (Lk < Lq, a length above
  * max_seqlen_*, a page id outside [0, num_pages), a bounded wait that ran
  * out) set an error word in the workspace and make the affected blocks skip
  * their work; fp2_get_status reads it.  Nothing prints, nothing throws.
@@ -108,7 +113,9 @@ typedef struct fp2_params {
 
 /* Offsets (bytes from params->workspace) of the intermediates, for callers
  * that read them (parity checks, exported masks).  Per-sequence regions are
- * padded to nqb_max = ceil(max_seqlen_q/B) query blocks and
+ * padded to nqb_max = min(floor((max_seqlen_q + 2B - 2)/B), nkb_max) query
+ * blocks (one more than ceil(max_seqlen_q/B) when a prefix that is not a
+ * multiple of B can shift a sequence's queries across a block boundary) and
  * nkb_max = ceil(max_seqlen_k/B) key blocks; nw = ceil(nkb_max/32). */
 typedef struct fp2_workspace_layout {
     size_t error_word;  /* uint32 [4]: first error code, detail */
@@ -173,7 +180,8 @@ fp2_status fp2_blockmean_cached(const void* k_cache, const void* v_cache,
                                 const fp2_params* params);
 
 /* Step 2 (abstract: instantaneous pattern discovery): pools each query block
- * (mean of its valid rows) and writes s_ij = qbar_i . kbar_j / sqrt(d) for
+ * (mean of the sequence's rows inside it; the first block of a sequence whose
+ * prefix is not a multiple of B holds only the rows from P on) and writes s_ij = qbar_i . kbar_j / sqrt(d) for
  * every causal j into the workspace scores.  Needs step 1. */
 fp2_status fp2_score(const void* q, const int32_t* cu_seqlens, int block, fp2_dtype dtype,
                      const fp2_params* params);

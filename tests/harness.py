@@ -63,16 +63,20 @@ def oracle_scores(inp: synth.Inputs):
 
 def pool_q_chunked(inp: synth.Inputs, b: int, chunk_blocks: int = 64):
     """Pooled queries of sequence b, computed block range by block range (so
-    a 128K sequence never needs all of Q in fp64 at once)."""
+    a 128K sequence never needs all of Q in fp64 at once).  Query blocks are
+    cut at absolute positions: with a prefix P, row t is in block
+    (P + t) // B - P // B."""
     B = inp.shape.B
     Lq = inp.shape.lens_q[b]
-    nqb = -(-Lq // B)
+    off = (inp.shape.lens_k[b] - Lq) % B
+    nqb = -(-(off + Lq) // B)
     parts = []
     a = int(inp.cu_seqlens_q[b])
     for i0 in range(0, nqb, chunk_blocks):
-        r0, r1 = i0 * B, min(Lq, (i0 + chunk_blocks) * B)
+        r0 = max(0, i0 * B - off)
+        r1 = min(Lq, (i0 + chunk_blocks) * B - off)
         Qc = inp._deq(inp.q[a + r0: a + r1], inp.q_scale)
-        parts.append(O.pool_q(Qc, B))
+        parts.append(O.pool_q(Qc, B, off if i0 == 0 else 0))
     return np.concatenate(parts, axis=1)
 
 

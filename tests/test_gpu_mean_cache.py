@@ -107,3 +107,49 @@ def test_bad_slot_is_reported():
                          pr.dtype, pr.params)
     st, det = fp2.get_status(pr.params)
     assert st == fp2.FP2_ERR_DEVICE_BOUNDS and det == 4
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_decode_steps_with_mean_cache(dtype):
+    """A 1000-token prefill chunk, then three decode steps (one query each).
+    Block 7 ends inside the first chunk (1000 = 7*128 + 104), so every step
+    re-averages it (it is not wholly inside the step's prefix) and writes it
+    back, while blocks 0-6 come from the cache.  Each step must equal the
+    uncached call bit for bit and the oracle within tolerance."""
+    first, steps = 1000, 3
+    total = first + steps
+    shape = H.small_shape([total], Hq=8, Hkv=2, dtype=dtype, page_size=64, seed=47)
+    inp = synth.make_inputs(shape)
+    nblk = -(-total // B)
+    table = torch.arange(nblk, dtype=torch.int32).reshape(1, nblk).cuda()
+    cache = torch.full((nblk, 2, shape.Hkv, shape.d), float("nan"), dtype=torch.float32,
+                       device="cuda")
+    c1 = chunk_problem(inp, [(0, first)], [first], [first])
+    fp2.prefill_cached(c1.q, c1.k, c1.v, c1.page_table, c1.cu_seqlens, 2.0, B, c1.dtype,
+                       c1.out, c1.params, table, nblk, cache, nblk)
+    c1.check()
+    K, V = inp.seq_k(0), inp.seq_v(0)
+    for st in range(steps):
+        pos = first + st
+        Lk = pos + 1
+        kbar, vbar, cnt = O.blockmean(K[:Lk], V[:Lk], B)
+        Qd = inp.seq_q(0)[pos:pos + 1]
+        Sd = O.score(O.pool_q(Qd, B, pos % B), kbar, pos // B)
+        tau = O.tau_for_drop([Sd], [pos // B], 0.5, guard=1e-3)
+        keep = O.mask(Sd, pos // B, tau)
+        assert keep.sum() < np.isfinite(Sd).sum()  # something is dropped
+        ref = O.attn_rows(Qd, K[:Lk], V[:Lk], kbar, vbar, cnt, keep, B,
+                          *O.all_rows(1, shape.Hq)).reshape(Qd.shape)
+        plain = chunk_problem(inp, [(pos, pos + 1)], [1], [Lk])
+        plain.prefill(tau)
+        plain.check()
+        step = chunk_problem(inp, [(pos, pos + 1)], [1], [Lk])
+        fp2.prefill_cached(step.q, step.k, step.v, step.page_table, step.cu_seqlens, tau, B,
+                           step.dtype, step.out, step.params, table, nblk, cache, nblk)
+        step.check()
+        assert torch.equal(step.out, plain.out)
+        L = step.layout()
+        a = step.ws_view("kbar", torch.float32, (1, shape.Hkv, L.nkb_max, shape.d))
+        e = plain.ws_view("kbar", torch.float32, (1, shape.Hkv, L.nkb_max, shape.d))
+        assert torch.equal(a, e)
+        H.assert_close(step.out.double().cpu().numpy(), ref, dtype == "fp8", f"step {st}")

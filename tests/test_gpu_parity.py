@@ -36,6 +36,19 @@ CASES = {
                                 dtype="fp8"),
     "chunk_prefix_short": dict(lens_q=[60, 128], lens_k=[512 + 60, 256 + 128], Hq=8, Hkv=2,
                                page_size=32),
+    # decode rows (Lq = 1) and chunks whose prefix is not a multiple of the
+    # block, mixed with ordinary prefill rows in one batch; prefixes 3000,
+    # 963, 1013, 127, 128, 0 (offsets 56, 67, 117, 127, 0, 0 into the block)
+    "mixed_decode_paged64": dict(lens_q=[1, 37, 700, 1, 1, 300],
+                                 lens_k=[3001, 1000, 1713, 128, 129, 300], Hq=8, Hkv=2,
+                                 page_size=64),
+    "mixed_decode_paged64_fp8": dict(lens_q=[1, 37, 700, 1, 1, 300],
+                                     lens_k=[3001, 1000, 1713, 128, 129, 300], Hq=8, Hkv=2,
+                                     page_size=64, dtype="fp8"),
+    "mixed_decode_g8": dict(lens_q=[1, 45, 250], lens_k=[777, 1000, 2503], Hq=16, Hkv=2),
+    "mixed_decode_g1": dict(lens_q=[1, 200, 5], lens_k=[2000, 1290, 133], Hq=4, Hkv=4),
+    "mixed_decode_b64_d64": dict(lens_q=[1, 90, 3], lens_k=[1500, 700, 67], Hq=4, Hkv=2, d=64,
+                                 B=64, page_size=16),
 }
 
 
@@ -142,7 +155,7 @@ def test_prefill_end_to_end(case):
 
 
 @pytest.mark.parametrize("name", ["tiny_1k_d64_b64", "varlen_paged64", "chunk_prefix_g8",
-                                  "ragged_2k_g4_fp8"])
+                                  "ragged_2k_g4_fp8", "mixed_decode_paged64", "mixed_decode_g1"])
 def test_keep_all_is_dense_attention(name):
     inp = make_inputs(name)
     pr = H.problem(inp)
@@ -197,22 +210,6 @@ def test_empty_sequence_in_batch():
 
 def test_device_errors_are_reported_not_faulted():
     inp = make_inputs("varlen_paged64")
-    # a prefix that is not a multiple of the block
-    pr = H.problem(inp)
-    bad = inp.seqlens_k.clone()
-    bad[1] += 5
-    bad_dev = bad.cuda()
-    pr.params.seqlens_k = bad_dev.data_ptr()
-    pr.params.max_seqlen_k = int(bad.max())
-    # workspace must be big enough for the larger max_seqlen_k
-    ws = torch.empty(fp2.workspace_size(pr.params, inp.shape.B), dtype=torch.uint8, device="cuda")
-    pr.params.workspace, pr.params.workspace_bytes = ws.data_ptr(), ws.numel()
-    pr.workspace = ws
-    fp2.workspace_init(pr.params)
-    pr.prefill(1.0)
-    st, det = fp2.get_status(pr.params)
-    assert st == fp2.FP2_ERR_UNSUPPORTED and det == 2
-    assert fp2.get_status(pr.params) == (fp2.FP2_OK, 0)  # cleared
     # a page id out of range
     pr2 = H.problem(inp)
     pt = pr2.page_table.clone()
@@ -221,6 +218,7 @@ def test_device_errors_are_reported_not_faulted():
     pr2.prefill(1.0)
     st, det = fp2.get_status(pr2.params)
     assert st == fp2.FP2_ERR_DEVICE_BOUNDS and det == 3
+    assert fp2.get_status(pr2.params) == (fp2.FP2_OK, 0)  # cleared
     # Lk < Lq
     pr3 = H.problem(inp)
     short = inp.seqlens_k.clone()
