@@ -257,6 +257,28 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         bool ok = true;
         for (int n = 0; n < n_items; ++n) {
             const int st = n & 1;
+            // the row's columns of this item, from shared memory, decided
+            // before S is waited for so the loads' latency hides behind it
+            const int item = items[n];
+            int lim = -1;                // real tile: last column taken
+            uint32_t dropped[BLK / 32];  // mean tile: the row's dropped blocks
+            if (item >= 0) {
+                const bool kept = row_ok && ((hb[item >> 5] >> (item & 31)) & 1u);
+                lim = !kept ? -1 : (item == iabs ? ppos - item * BLK : BLK - 1);
+            } else {
+                const int tv = -item - 1;
+#pragma unroll
+                for (int w = 0; w < BLK / 32; ++w) {
+                    const int j0 = tv * BLK + w * 32;  // multiple of 32
+                    uint32_t dm = 0u;
+                    if (row_ok && j0 < iabs) {
+                        dm = ~hb[j0 >> 5];
+                        const int nvalid = iabs - j0;
+                        if (nvalid < 32) dm &= (1u << nvalid) - 1u;
+                    }
+                    dropped[w] = dm;
+                }
+            }
             if (!__all_sync(0xffffffffu,
                             mbar_wait(&bars[B_S_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs))) {
                 set_error(p.err, kErrTimeout, kDetWaitBase + 4);
@@ -272,12 +294,8 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             tc_fence_before();
             mbar_arrive(&bars[B_S_FREE + st]);
 
-            const int item = items[n];
             float mx = -INFINITY;
             if (item >= 0) {
-                const int j = item;
-                const bool kept = row_ok && ((hb[j >> 5] >> (j & 31)) & 1u);
-                const int lim = !kept ? -1 : (j == iabs ? ppos - j * BLK : BLK - 1);
 #pragma unroll
                 for (int c = 0; c < BLK; ++c) {
                     const float v = c <= lim ? x[c] * sl2 : -INFINITY;
@@ -285,23 +303,15 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                     mx = fmaxf(mx, v);
                 }
             } else {
-                const int tv = -item - 1;
 #pragma unroll
-                for (int c0 = 0; c0 < BLK; c0 += 32) {
-                    const int j0 = tv * BLK + c0;  // multiple of 32
-                    uint32_t dropped = 0u;
-                    if (row_ok && j0 < iabs) {
-                        dropped = ~hb[j0 >> 5];
-                        const int nvalid = iabs - j0;
-                        if (nvalid < 32) dropped &= (1u << nvalid) - 1u;
-                    }
+                for (int w = 0; w < BLK / 32; ++w)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const float v = ((dropped >> e) & 1u) ? fmaf(x[c0 + e], sl2, lb) : -INFINITY;
-                        x[c0 + e] = v;
+                        const float v = ((dropped[w] >> e) & 1u) ? fmaf(x[w * 32 + e], sl2, lb)
+                                                                : -INFINITY;
+                        x[w * 32 + e] = v;
                         mx = fmaxf(mx, v);
                     }
-                }
             }
             float alpha = 1.f;
             bool rescale = false;

@@ -281,6 +281,35 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int n = 0; n < n_items; ++n) {
+            // Which columns of this item the row takes: decided from shared
+            // memory before S is waited for, so those loads' latency hides
+            // behind the wait.  Masks act on raw scores (the scale sl2 is
+            // positive); the bias of a mean tile (log2 n_j) and the running
+            // max fold into the one FFMA that feeds exp2:
+            //   p = 2^(x * sl2 + (bias - m)).
+            const int item = items[n];
+            bool live;                  // this row takes part in this item
+            float bias = 0.f;
+            uint32_t dropped[BLK / 32];  // mean tiles: the row's dropped blocks
+            if (item >= 0) {
+                live = row_ok && ((hb[item >> 5] >> (item & 31)) & 1u);
+            } else {
+                const int tv = -item - 1;
+                bias = lb;
+                live = false;
+#pragma unroll
+                for (int w = 0; w < BLK / 32; ++w) {
+                    const int j0 = tv * BLK + w * 32;
+                    uint32_t dm = 0u;
+                    if (row_ok && j0 < iabs) {
+                        dm = ~hb[j0 >> 5];
+                        const int nvalid = iabs - j0;
+                        if (nvalid < 32) dm &= (1u << nvalid) - 1u;
+                    }
+                    dropped[w] = dm;
+                    live |= dm != 0u;
+                }
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[PB_S_FULL + X], n & 1, abort_flag,
                                                    kWaitLimitNs))) {
                 set_error(p.err, kErrTimeout, kDetWaitBase + 4);
@@ -294,38 +323,18 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             for (int c = 0; c < BLK / 32; ++c) tmem_ld32f(s_addr + c * 32, x + c * 32);
             tmem_wait_ld();
 
-            const int item = items[n];
-            // Masks act on raw scores (the scale sl2 is positive); the bias
-            // of a mean tile (log2 n_j) and the running max fold into the one
-            // FFMA that feeds exp2:  p = 2^(x * sl2 + (bias - m)).
-            bool live;       // this row takes part in this item
-            float bias = 0.f;
             if (item >= 0) {
-                const int j = item;
-                live = row_ok && ((hb[j >> 5] >> (j & 31)) & 1u);
-                if (live && j == iabs) {
-                    const int lim = ppos - j * BLK;
+                if (live && item == iabs) {
+                    const int lim = ppos - item * BLK;
 #pragma unroll
                     for (int c = 0; c < BLK; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
                 }
             } else {
-                const int tv = -item - 1;
-                bias = lb;
-                live = false;
 #pragma unroll
-                for (int c0 = 0; c0 < BLK; c0 += 32) {
-                    const int j0 = tv * BLK + c0;
-                    uint32_t dropped = 0u;
-                    if (row_ok && j0 < iabs) {
-                        dropped = ~hb[j0 >> 5];
-                        const int nvalid = iabs - j0;
-                        if (nvalid < 32) dropped &= (1u << nvalid) - 1u;
-                    }
-                    live |= dropped != 0u;
+                for (int w = 0; w < BLK / 32; ++w)
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        x[c0 + e] = ((dropped >> e) & 1u) ? x[c0 + e] : -INFINITY;
-                }
+                        x[w * 32 + e] = ((dropped[w] >> e) & 1u) ? x[w * 32 + e] : -INFINITY;
             }
             float mx = -INFINITY;
             if (live) {
