@@ -80,6 +80,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
     const uint32_t raw_s = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
+    const uint32_t q_s = sbase + C::OFF_Q;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
@@ -110,6 +111,13 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             mbar_init(&bars[k], (k == PB_P_READY || k == PB_P_READY + 1) ? 128u : 1u);
         misc[1] = 0;
         fence_mbar_init();
+        // both Q tiles right away: their latency overlaps the kept-bit loads
+        // and the item list
+        mbar_arrive_expect_tx(&bars[PB_Q_FULL], 2 * C::Q_BYTES);
+        for (int x = 0; x < 2; ++x)
+            for (int c = 0; c < C::NCH; ++c)
+                tma_load_3d(q_s + x * C::Q_BYTES + c * (128 * 128), &maps.q, &bars[PB_Q_FULL],
+                            c * C::CH, hk * G, s.q0 + t_begin + x * TOK);
     }
     if (warp == 9) {
         tmem_alloc(&misc[0], 512);
@@ -126,7 +134,6 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
     tc_fence_after();
     const uint32_t tmem = misc[0];
     const int n_items = (int)misc[2];
-    const uint32_t q_s = sbase + C::OFF_Q;
 
     if (warp >= 8) {
       regs_decrease<56>();
@@ -136,14 +143,8 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         // and issues every copy
         int* pring = reinterpret_cast<int*>(smem + C::OFF_RING);
         if (lane == 0) {
-            prefetch_tmap(&maps.q);
             prefetch_tmap(&maps.k);
             prefetch_tmap(&maps.v);
-            mbar_arrive_expect_tx(&bars[PB_Q_FULL], 2 * C::Q_BYTES);
-            for (int x = 0; x < 2; ++x)
-                for (int c = 0; c < C::NCH; ++c)
-                    tma_load_3d(q_s + x * C::Q_BYTES + c * (128 * 128), &maps.q, &bars[PB_Q_FULL],
-                                c * C::CH, hk * G, s.q0 + t_begin + x * TOK);
         }
         // K runs one item ahead of V: iteration n loads K(n), then V(n-1)
         int k_issued = 0, v_issued = 0;

@@ -43,7 +43,8 @@
  *    k_scale [Hkv], v_scale [Hkv] (fp32, device).  out is bf16 unless
  *    params->out_dtype asks for e4m3.
  *  - Base pointers of q, k_cache, v_cache and out must be 16-byte aligned.
- *  - Supported: head_dim 64 or 128 (FP8: 128), block 64 or 128,
+ *  - Supported: head_dim 64 or 128, block 64 or 128 (FP8: head_dim 128
+ *    and block 128 only; other FP8 shapes return FP2_ERR_UNSUPPORTED),
  *    G = Hq/Hkv in {1,2,4,8} with 128/G <= block, page_size a power of two
  *    in [16, 256] that divides the block or is divided by it.
  *
