@@ -49,6 +49,8 @@ def parse():
                     help="one mask per KV group (variant) instead of one per query head")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="query-block chunks of the host-buffer pipeline (1..16)")
     ap.add_argument("--no-dense", action="store_true")
     return ap.parse_args()
 
@@ -297,31 +299,38 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
 
         e2e = None
         if not args.no_e2e:
-            # through the public API with HOST buffers: H2D of q, k, v from
-            # pinned memory, fp2_prefill, D2H of the output, every step
+            # through the public API with HOST buffers: fp2_prefill_host
+            # uploads q, K, V from pinned memory and downloads the output
+            # every step, the copies pipelined with the kernels over
+            # query-block chunks on two copy streams
             hq = inp.q.pin_memory()
             hk = inp.k.pin_memory()
             hv = inp.v.pin_memory()
             hout = torch.empty(pr.out.shape, dtype=pr.out.dtype).pin_memory()
+            cu_h = inp.cu_seqlens_q.to(torch.int32).contiguous()
+            lk_h = inp.seqlens_k.to(torch.int32).contiguous()
+            up, down = torch.cuda.Stream(), torch.cuda.Stream()
+            io = fp2.host_io(hq, hk, hv, hout, q, k, v, pr.out, cu_h, lk_h, upload_stream=up,
+                             download_stream=down, num_chunks=args.e2e_chunks)
             nsteps = max(2, min(args.steps, 5))
             for it in range(nsteps + 1):
                 if it == 1:
                     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     ea.record(stream)
-                q.copy_(hq, non_blocking=True)
-                k.copy_(hk, non_blocking=True)
-                v.copy_(hv, non_blocking=True)
-                fp2.prefill(q, k, v, pt, cu, tau, B, dt, pr.out, P)
-                hout.copy_(pr.out, non_blocking=True)
+                # each call leaves `stream` waiting for its last download
+                fp2.prefill_host(io, pt, cu, tau, B, dt, P)
             eb.record(stream)
             stream.synchronize()
+            torch.cuda.synchronize()
             pr.check()
             e2e_ms = ea.elapsed_time(eb) / nsteps
             e2e = {"value": e2e_ms, "unit": "ms/layer",
                    "h2d_bytes_per_step": int(hq.numel() * hq.element_size() +
                                              hk.numel() * hk.element_size() +
                                              hv.numel() * hv.element_size()),
-                   "d2h_bytes_per_step": int(hout.numel() * hout.element_size())}
+                   "d2h_bytes_per_step": int(hout.numel() * hout.element_size()),
+                   "path": f"fp2_prefill_host, {args.e2e_chunks} query-block chunks, pinned host "
+                           "buffers, upload and download streams"}
         mean_cache = None
         prefixes = [Lk - Lq for Lq, Lk in zip(s.lens_q, s.lens_k)]
         if inp.paged and max(prefixes) > 0:

@@ -1,9 +1,10 @@
 // fp2_api.cu -- the C ABI of include/fp2.h: argument validation, workspace
-// layout, stream-ordered launches of the four kernels, status read-back and
-// the host-side tau calibration utility.
+// layout, stream-ordered launches of the four kernels, the host-buffer
+// pipeline, status read-back and the host-side tau calibration utility.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "fp2.h"
@@ -119,6 +120,8 @@ fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_
     kp.nqb_max = L.nqb_max;
     kp.nkb_max = L.nkb_max;
     kp.nw = L.nw;
+    kp.qb_lo = 0;
+    kp.qb_n = L.nqb_max;
     kp.fp8 = dtype == FP2_FP8_E4M3;
     kp.uses_kv = uses_kv ? 1 : 0;
     kp.group_masks = P->group_masks ? 1 : 0;
@@ -146,6 +149,26 @@ fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_
 cudaStream_t stream_of(const fp2_params* P) { return static_cast<cudaStream_t>(P->stream); }
 
 fp2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP2_OK : FP2_ERR_CUDA; }
+
+// Events that order fp2_prefill_host's three streams: created once per device
+// on first use, re-recorded by every call while g_host_mutex is held (so a
+// record and the waits on it are never interleaved with another call's).
+constexpr int kHostMaxChunks = 16;
+constexpr int kHostEvents = 2 * kHostMaxChunks + 3;
+constexpr int kHostMaxDevices = 64;
+struct HostEvents {
+    bool ready = false;
+    cudaEvent_t ev[kHostEvents];
+};
+std::mutex g_host_mutex;
+HostEvents g_host_events[kHostMaxDevices];
+
+// `to` waits for the work queued so far on `from` (nothing when they are one stream)
+cudaError_t join(cudaStream_t from, cudaStream_t to, cudaEvent_t e) {
+    if (from == to) return cudaSuccess;
+    cudaError_t r = cudaEventRecord(e, from);
+    return r != cudaSuccess ? r : cudaStreamWaitEvent(to, e, 0);
+}
 
 }  // namespace
 
@@ -386,6 +409,104 @@ fp2_status fp2_calibrate_tau(const int32_t* cu_seqlens, int block, float target_
     const double lo = *std::max_element(margins.begin(), margins.begin() + k);
     *tau_out = (float)(0.5 * (lo + hi));
     return FP2_OK;
+}
+
+fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
+                            const int32_t* cu_seqlens, float tau, int block, fp2_dtype dtype,
+                            const fp2_params* params) {
+    if (!io || !params) return FP2_ERR_INVALID_ARG;
+    if (io->num_chunks < 1 || io->num_chunks > kHostMaxChunks) return FP2_ERR_INVALID_ARG;
+    if (!io->q_host || !io->k_host || !io->v_host || !io->out_host || !io->q_dev ||
+        !io->k_dev || !io->v_dev || !io->out_dev || !io->cu_seqlens_host)
+        return FP2_ERR_INVALID_ARG;
+    if (params->seqlens_k && !io->seqlens_k_host) return FP2_ERR_INVALID_ARG;
+    KParams kp;
+    fp2_status st = prepare(params, block, dtype, cu_seqlens, page_table, kp);
+    if (st != FP2_OK) return st;
+    if (!aligned16(io->q_dev) || !aligned16(io->k_dev) || !aligned16(io->v_dev) ||
+        !aligned16(io->out_dev))
+        return FP2_ERR_INVALID_ARG;
+    if (std::isnan(tau)) return FP2_ERR_INVALID_ARG;
+    if (kp.total_q == 0) return FP2_OK;
+    if (!page_table && kp.total_k == 0) return FP2_ERR_INVALID_ARG;
+
+    // per-sequence geometry from the host copies of the lengths
+    const int S = kp.num_seqs;
+    const int32_t* cu = io->cu_seqlens_host;
+    std::vector<int> q0(S), Lq(S), off(S);
+    for (int b = 0; b < S; ++b) {
+        q0[b] = cu[b];
+        Lq[b] = cu[b + 1] - cu[b];
+        const int Lk = io->seqlens_k_host ? io->seqlens_k_host[b] : Lq[b];
+        if (q0[b] < 0 || Lq[b] < 0 || Lq[b] > kp.max_seqlen_q || Lk < Lq[b] ||
+            Lk > kp.max_seqlen_k || q0[b] + Lq[b] > kp.total_q)
+            return FP2_ERR_INVALID_ARG;
+        off[b] = (Lk - Lq[b]) % block;
+    }
+    const size_t elt_in = kp.fp8 ? 1 : 2, elt_out = kp.out_fp8 ? 1 : 2;
+    const size_t row_in = (size_t)kp.Hq * kp.d * elt_in, row_out = (size_t)kp.Hq * kp.d * elt_out;
+    const size_t kv_bytes = (page_table ? (size_t)kp.num_pages * kp.page_size : (size_t)kp.total_k) *
+                            kp.Hkv * kp.d * elt_in;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP2_ERR_CUDA;
+    if (dev < 0 || dev >= kHostMaxDevices) return FP2_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_host_mutex);
+    HostEvents& pool = g_host_events[dev];
+    if (!pool.ready) {
+        for (int e = 0; e < kHostEvents; ++e)
+            if (cudaEventCreateWithFlags(&pool.ev[e], cudaEventDisableTiming) != cudaSuccess)
+                return FP2_ERR_CUDA;
+        pool.ready = true;
+    }
+    cudaEvent_t* ev = pool.ev;
+    cudaStream_t s = stream_of(params);
+    cudaStream_t up = io->upload_stream ? static_cast<cudaStream_t>(io->upload_stream) : s;
+    cudaStream_t down = io->download_stream ? static_cast<cudaStream_t>(io->download_stream) : s;
+    auto* qh = static_cast<const uint8_t*>(io->q_host);
+    auto* qd = static_cast<uint8_t*>(io->q_dev);
+    auto* oh = static_cast<uint8_t*>(io->out_host);
+    auto* od = static_cast<const uint8_t*>(io->out_dev);
+
+    // K and V whole (any key block may be kept or averaged), then the means
+    cudaError_t e = join(s, up, ev[0]);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(io->k_dev, io->k_host, kv_bytes, cudaMemcpyHostToDevice, up);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(io->v_dev, io->v_host, kv_bytes, cudaMemcpyHostToDevice, up);
+    if (e == cudaSuccess) e = join(up, s, ev[1]);
+    if (e == cudaSuccess) e = fp2::launch_blockmean(kp, io->k_dev, io->v_dev, s);
+    // query-block ranges, highest (longest rows) first
+    const int per = (kp.nqb_max + io->num_chunks - 1) / io->num_chunks;
+    for (int c = 0; e == cudaSuccess && c < io->num_chunks; ++c) {
+        const int hi = kp.nqb_max - c * per, lo = std::max(0, hi - per);
+        if (hi <= 0) break;
+        // the sequences' query rows of blocks [lo, hi): rows t with
+        // lo <= (off + t) / B < hi
+        for (int b = 0; e == cudaSuccess && b < S; ++b) {
+            const int r0 = std::max(0, lo * block - off[b]);
+            const int r1 = std::min(Lq[b], hi * block - off[b]);
+            if (r1 > r0)
+                e = cudaMemcpyAsync(qd + (size_t)(q0[b] + r0) * row_in, qh + (size_t)(q0[b] + r0) * row_in,
+                                    (size_t)(r1 - r0) * row_in, cudaMemcpyHostToDevice, up);
+        }
+        if (e == cudaSuccess) e = join(up, s, ev[2 + 2 * c]);
+        kp.qb_lo = lo;
+        kp.qb_n = hi - lo;
+        if (e == cudaSuccess) e = fp2::launch_score(kp, io->q_dev, s);
+        if (e == cudaSuccess) e = fp2::launch_mask(kp, tau, s);
+        if (e == cudaSuccess)
+            e = fp2::launch_attn(kp, io->q_dev, io->k_dev, io->v_dev, kp.kept_bits, io->out_dev, s);
+        if (e == cudaSuccess) e = join(s, down, ev[3 + 2 * c]);
+        for (int b = 0; e == cudaSuccess && b < S; ++b) {
+            const int r0 = std::max(0, lo * block - off[b]);
+            const int r1 = std::min(Lq[b], hi * block - off[b]);
+            if (r1 > r0)
+                e = cudaMemcpyAsync(oh + (size_t)(q0[b] + r0) * row_out, od + (size_t)(q0[b] + r0) * row_out,
+                                    (size_t)(r1 - r0) * row_out, cudaMemcpyDeviceToHost, down);
+        }
+    }
+    // params->stream ends after the last download
+    if (e == cudaSuccess) e = join(down, s, ev[kHostEvents - 1]);
+    return cuda_status(e);
 }
 
 }  // extern "C"

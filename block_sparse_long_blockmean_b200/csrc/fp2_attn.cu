@@ -86,7 +86,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
     const int ntq = BLK / TOK;
     // longest-first order: the largest query block index goes first
     const int per_i = p.num_seqs * p.Hkv * ntq;
-    const int i = p.nqb_max - 1 - (int)(blockIdx.x / per_i);
+    const int i = p.qb_lo + p.qb_n - 1 - (int)(blockIdx.x / per_i);
     const int rem = (int)(blockIdx.x % per_i);
     const int b = rem / (p.Hkv * ntq);
     const int hk = (rem / ntq) % p.Hkv;
@@ -546,7 +546,7 @@ static cudaError_t launch_attn_t(const KParams& p, const void* q, const void* k,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int ntq = BLK / TOK;
-    const long long grid = (long long)p.nqb_max * p.num_seqs * p.Hkv * ntq;
+    const long long grid = (long long)p.qb_n * p.num_seqs * p.Hkv * ntq;
     if (grid <= 0) return cudaSuccess;
     attn_kernel<D, BLK, FP8><<<(unsigned)grid, 192, smem, st>>>(
         p, maps, kept_bits, static_cast<__nv_bfloat16*>(out), items_cap);

@@ -91,7 +91,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
     const int TOK = 128 / G;
     const int npair = BLK / (2 * TOK);
     const int per_i = p.num_seqs * p.Hkv * npair;
-    const int i = p.nqb_max - 1 - (int)(blockIdx.x / per_i);  // longest first
+    const int i = p.qb_lo + p.qb_n - 1 - (int)(blockIdx.x / per_i);  // longest first
     const int rem = (int)(blockIdx.x % per_i);
     const int b = rem / (p.Hkv * npair);
     const int hk = (rem / npair) % p.Hkv;
@@ -508,7 +508,7 @@ cudaError_t launch_attn_pair_t(const KParams& p, const void* q, const void* k, c
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int npair = BLK / (2 * TOK);
-    const long long grid = (long long)p.nqb_max * p.num_seqs * p.Hkv * npair;
+    const long long grid = (long long)p.qb_n * p.num_seqs * p.Hkv * npair;
     if (grid <= 0) return cudaSuccess;
     attn_pair_kernel<D, BLK, FP8><<<(unsigned)grid, 384, smem, st>>>(
         p, maps, kept_bits, static_cast<__nv_bfloat16*>(out), items_cap);

@@ -15,6 +15,9 @@ struct KParams {
     int paged, page_size, max_pages, num_pages;
     int max_seqlen_q, max_seqlen_k;
     int nqb_max, nkb_max, nw;
+    // query blocks [qb_lo, qb_lo + qb_n) of every sequence are processed by
+    // the score, mask and attention launches (all of them: 0, nqb_max)
+    int qb_lo, qb_n;
     int fp8;
     int uses_kv;               // 0: the launch never reads K/V (no key-extent check)
     int group_masks;           // score every head with its group's mean pooled query

@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
     __shared__ float red[TPP][G * D];
     __shared__ float qb[G * D];
 
-    const int i = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int i = p.qb_lo + (int)blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
     if (i >= s.nqb) return;
@@ -311,11 +311,13 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
 // Emits the kept bitmask (all nw words), the ascending kept list and count.
 __global__ void __launch_bounds__(128) mask_kernel(KParams p, float tau) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long row = (long long)blockIdx.x * 4 + warp;
-    const long long nrows = (long long)p.num_seqs * p.Hq * p.nqb_max;
-    if (row >= nrows) return;
-    const int i = (int)(row % p.nqb_max);
-    const int b = (int)(row / ((long long)p.nqb_max * p.Hq));
+    // rows of this launch: (sequence, head) x query blocks [qb_lo, qb_lo + qb_n)
+    const long long r = (long long)blockIdx.x * 4 + warp;
+    if (r >= (long long)p.num_seqs * p.Hq * p.qb_n) return;
+    const int i = p.qb_lo + (int)(r % p.qb_n);
+    const long long bh = r / p.qb_n;  // b * Hq + h
+    const int b = (int)(bh / p.Hq);
+    const long long row = bh * p.nqb_max + i;  // [S][Hq][nqb_max] index
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
     if (i >= s.nqb) return;
@@ -368,7 +370,8 @@ static void score_dispatch_g(const KParams& p, const uint8_t* Q, dim3 grid, cuda
 }
 
 cudaError_t launch_score(const KParams& p, const void* q, cudaStream_t st) {
-    dim3 grid(p.nqb_max, p.Hkv, p.num_seqs);
+    dim3 grid(p.qb_n, p.Hkv, p.num_seqs);
+    if (p.qb_n <= 0) return cudaSuccess;
     auto Q = static_cast<const uint8_t*>(q);
     if (p.fp8) {
         if (p.d == 128) score_dispatch_g<128, true>(p, Q, grid, st);
@@ -381,7 +384,8 @@ cudaError_t launch_score(const KParams& p, const void* q, cudaStream_t st) {
 }
 
 cudaError_t launch_mask(const KParams& p, float tau, cudaStream_t st) {
-    const long long rows = (long long)p.num_seqs * p.Hq * p.nqb_max;
+    const long long rows = (long long)p.num_seqs * p.Hq * p.qb_n;
+    if (rows <= 0) return cudaSuccess;
     const unsigned blocks = (unsigned)((rows + 3) / 4);
     mask_kernel<<<blocks, 128, 0, st>>>(p, tau);
     return cudaGetLastError();

@@ -81,6 +81,26 @@ class WorkspaceLayout(ctypes.Structure):
     ]
 
 
+class HostIO(ctypes.Structure):
+    """Mirror of ``fp2_host_io`` (host buffers, their device twins, the copy
+    streams and the number of query-block chunks of fp2_prefill_host)."""
+    _fields_ = [
+        ("q_host", ctypes.c_void_p),
+        ("k_host", ctypes.c_void_p),
+        ("v_host", ctypes.c_void_p),
+        ("out_host", ctypes.c_void_p),
+        ("q_dev", ctypes.c_void_p),
+        ("k_dev", ctypes.c_void_p),
+        ("v_dev", ctypes.c_void_p),
+        ("out_dev", ctypes.c_void_p),
+        ("cu_seqlens_host", ctypes.c_void_p),
+        ("seqlens_k_host", ctypes.c_void_p),
+        ("upload_stream", ctypes.c_void_p),
+        ("download_stream", ctypes.c_void_p),
+        ("num_chunks", ctypes.c_int),
+    ]
+
+
 _LIB = None
 _VP = ctypes.c_void_p
 _PP = ctypes.POINTER(Params)
@@ -96,6 +116,8 @@ SIGNATURES = {
     "fp2_prefill_cached": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, ctypes.c_float, ctypes.c_int,
                                           ctypes.c_int, _VP, _PP, _VP, ctypes.c_int, _VP,
                                           ctypes.c_int]),
+    "fp2_prefill_host": (ctypes.c_int, [ctypes.POINTER(HostIO), _VP, _VP, ctypes.c_float,
+                                        ctypes.c_int, ctypes.c_int, _PP]),
     "fp2_blockmean": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, ctypes.c_int, _PP]),
     "fp2_blockmean_cached": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, ctypes.c_int, _VP,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, _PP]),
@@ -174,6 +196,34 @@ def prefill_noalloc(q, k_cache, v_cache, page_table, cu_seqlens, tau: float, blo
     _check(lib().fp2_prefill_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
                                      _ptr(cu_seqlens), float(tau), block, dtype, _ptr(out),
                                      ctypes.byref(params)), "fp2_prefill_noalloc")
+
+
+def prefill_host(io: HostIO, page_table, cu_seqlens, tau: float, block: int, dtype: int,
+                 params: Params) -> None:
+    """fp2_prefill with q, K/V and out in (pinned) host memory, copies
+    pipelined with the kernels over ``io.num_chunks`` query-block ranges.
+    ``io`` holds raw pointers; the caller keeps the tensors behind them alive
+    until ``params.stream`` has been synchronised."""
+    _check(lib().fp2_prefill_host(ctypes.byref(io), _ptr(page_table), _ptr(cu_seqlens),
+                                  float(tau), block, dtype, ctypes.byref(params)),
+           "fp2_prefill_host")
+
+
+def host_io(q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_dev, cu_seqlens_host,
+            seqlens_k_host=None, upload_stream=None, download_stream=None,
+            num_chunks: int = 8) -> HostIO:
+    """An ``fp2_host_io`` from tensors (host ones on the CPU, ideally pinned;
+    int32 length arrays on the CPU) and torch streams (or None)."""
+    io = HostIO()
+    io.q_host, io.k_host, io.v_host, io.out_host = (_ptr(q_host), _ptr(k_host), _ptr(v_host),
+                                                    _ptr(out_host))
+    io.q_dev, io.k_dev, io.v_dev, io.out_dev = _ptr(q_dev), _ptr(k_dev), _ptr(v_dev), _ptr(out_dev)
+    io.cu_seqlens_host = _ptr(cu_seqlens_host)
+    io.seqlens_k_host = _ptr(seqlens_k_host)
+    io.upload_stream = upload_stream.cuda_stream if upload_stream is not None else None
+    io.download_stream = download_stream.cuda_stream if download_stream is not None else None
+    io.num_chunks = int(num_chunks)
+    return io
 
 
 def blockmean(k_cache, v_cache, page_table, cu_seqlens, block: int, dtype: int,

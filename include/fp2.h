@@ -220,6 +220,55 @@ fp2_status fp2_get_status(const fp2_params* params, uint32_t* detail);
 fp2_status fp2_calibrate_tau(const int32_t* cu_seqlens, int block, float target_drop,
                              const fp2_params* params, float* tau_out);
 
+/* Host-resident inputs and outputs of fp2_prefill_host.  Every pointer is
+ * caller-owned; the library allocates nothing.  Host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister): pageable memory works but its copies do
+ * not overlap the kernels. */
+typedef struct fp2_host_io {
+    const void* q_host;   /* [total_q, Hq, d] q (bf16 or e4m3, as dtype) */
+    const void* k_host;   /* the whole K cache, the layout k_cache has in fp2_prefill:
+                             [total_k, Hkv, d] or [num_pages, page_size, Hkv, d] */
+    const void* v_host;   /* the whole V cache, same layout */
+    void* out_host;       /* [total_q, Hq, d], bf16 or e4m3 (params->out_dtype) */
+    void* q_dev;          /* device buffers of the same sizes, 16-byte aligned */
+    void* k_dev;
+    void* v_dev;
+    void* out_dev;
+    const int32_t* cu_seqlens_host; /* host copy of cu_seqlens [num_seqs+1] */
+    const int32_t* seqlens_k_host;  /* host copy of params->seqlens_k [num_seqs],
+                                       NULL when params->seqlens_k is NULL */
+    void* upload_stream;   /* cudaStream_t for the host->device copies; NULL:
+                              params->stream (no overlap) */
+    void* download_stream; /* cudaStream_t for the device->host copies; NULL:
+                              params->stream (no overlap) */
+    int num_chunks;        /* query-block chunks of the pipeline, 1..16 */
+} fp2_host_io;
+
+/* fp2_prefill with q, K/V and out in host memory: the call a serving process
+ * makes when the layer's inputs are not yet on the GPU (packaging of the
+ * same method, not a step of it).  It uploads K and V and averages every
+ * key block, then runs score, mask and attention over num_chunks ranges of
+ * query blocks (highest first), uploading each range's query rows while the
+ * previous range computes and downloading each range's output rows while
+ * the next one computes.  Results are bit-identical to fp2_prefill on the
+ * same data.
+ *  - Queues work on params->stream, io->upload_stream and
+ *    io->download_stream and returns; params->stream is made to wait for the
+ *    last download, so synchronising params->stream means out_host is done.
+ *    The uploads first wait for work already queued on params->stream, so
+ *    back-to-back calls on the same device buffers do not race.
+ *  - cu_seqlens, params->seqlens_k and page_table stay device arrays (small,
+ *    usually resident); cu_seqlens_host / seqlens_k_host must hold the same
+ *    values (they place each range's query rows).
+ *  - Uses a library-owned pool of CUDA events per device, created on the
+ *    first call (make it before any stream capture); calls from several
+ *    host threads are serialised while they queue.
+ *  - Errors as fp2_prefill; io == NULL, a NULL buffer, num_chunks outside
+ *    [1, 16] or misaligned device buffers return FP2_ERR_INVALID_ARG. */
+fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
+                            const int32_t* cu_seqlens, float tau, int block, fp2_dtype dtype,
+                            const fp2_params* params);
+
 /* Bytes of the library-owned device scratch used by fp2_prefill_noalloc. */
 #define FP2_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -49,11 +49,14 @@ def test_every_declared_symbol_is_exported(lib):
 def test_struct_layout_matches_header(tmp_path):
     fields = [f for f, _ in fp2.Params._fields_]
     lfields = [f for f, _ in fp2.WorkspaceLayout._fields_]
+    hfields = [f for f, _ in fp2.HostIO._fields_]
     prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "fp2.h"', "int main(void){",
             'printf("%zu\\n", sizeof(fp2_params));']
     prog += [f'printf("%zu\\n", offsetof(fp2_params, {f}));' for f in fields]
     prog += ['printf("%zu\\n", sizeof(fp2_workspace_layout));']
     prog += [f'printf("%zu\\n", offsetof(fp2_workspace_layout, {f}));' for f in lfields]
+    prog += ['printf("%zu\\n", sizeof(fp2_host_io));']
+    prog += [f'printf("%zu\\n", offsetof(fp2_host_io, {f}));' for f in hfields]
     prog += ["return 0;}"]
     c = tmp_path / "probe.c"
     c.write_text("\n".join(prog))
@@ -65,6 +68,8 @@ def test_struct_layout_matches_header(tmp_path):
     want = [ctypes.sizeof(fp2.Params)] + [getattr(fp2.Params, f).offset for f in fields]
     want += [ctypes.sizeof(fp2.WorkspaceLayout)]
     want += [getattr(fp2.WorkspaceLayout, f).offset for f in lfields]
+    want += [ctypes.sizeof(fp2.HostIO)]
+    want += [getattr(fp2.HostIO, f).offset for f in hfields]
     assert vals == want
 
 
@@ -170,3 +175,30 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(fp2, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(ImportError):
         fp2.lib()
+
+
+def test_host_pipeline_rejects_bad_arguments_before_any_cuda_work(lib):
+    P = base_params()
+    fake = 1 << 20  # never dereferenced
+    assert lib.fp2_prefill_host(None, None, fake, 1.0, 128, 0, ctypes.byref(P)) == \
+        fp2.FP2_ERR_INVALID_ARG
+    io = fp2.HostIO()
+    for f, _ in fp2.HostIO._fields_:
+        if f not in ("seqlens_k_host", "upload_stream", "download_stream", "num_chunks"):
+            setattr(io, f, fake)
+    for chunks in (0, 17, -1):
+        io.num_chunks = chunks
+        assert lib.fp2_prefill_host(ctypes.byref(io), None, fake, 1.0, 128, 0,
+                                    ctypes.byref(P)) == fp2.FP2_ERR_INVALID_ARG
+    io.num_chunks = 4
+    io.out_host = None
+    assert lib.fp2_prefill_host(ctypes.byref(io), None, fake, 1.0, 128, 0,
+                                ctypes.byref(P)) == fp2.FP2_ERR_INVALID_ARG
+    io.out_host = fake
+    P.seqlens_k = fake  # device lengths given but no host copy of them
+    assert lib.fp2_prefill_host(ctypes.byref(io), None, fake, 1.0, 128, 0,
+                                ctypes.byref(P)) == fp2.FP2_ERR_INVALID_ARG
+    P.seqlens_k = None
+    # no workspace: the same validation as fp2_prefill
+    assert lib.fp2_prefill_host(ctypes.byref(io), None, fake, 1.0, 128, 0,
+                                ctypes.byref(P)) == fp2.FP2_ERR_WORKSPACE
