@@ -309,9 +309,11 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
             hout = torch.empty(pr.out.shape, dtype=pr.out.dtype).pin_memory()
             cu_h = inp.cu_seqlens_q.to(torch.int32).contiguous()
             lk_h = inp.seqlens_k.to(torch.int32).contiguous()
+            cuk_h = None if inp.paged else inp.cu_seqlens_k.to(torch.int32).contiguous()
             up, down = torch.cuda.Stream(), torch.cuda.Stream()
             io = fp2.host_io(hq, hk, hv, hout, q, k, v, pr.out, cu_h, lk_h, upload_stream=up,
-                             download_stream=down, num_chunks=args.e2e_chunks)
+                             download_stream=down, num_chunks=args.e2e_chunks,
+                             cu_seqlens_k_host=cuk_h)
             nsteps = max(2, min(args.steps, 5))
             for it in range(nsteps + 1):
                 if it == 1:

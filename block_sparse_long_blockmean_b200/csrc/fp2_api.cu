@@ -122,6 +122,8 @@ fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_
     kp.nw = L.nw;
     kp.qb_lo = 0;
     kp.qb_n = L.nqb_max;
+    kp.kb_lo = 0;
+    kp.kb_n = L.nkb_max;
     kp.fp8 = dtype == FP2_FP8_E4M3;
     kp.uses_kv = uses_kv ? 1 : 0;
     kp.group_masks = P->group_masks ? 1 : 0;
@@ -432,21 +434,27 @@ fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
 
     // per-sequence geometry from the host copies of the lengths
     const int S = kp.num_seqs;
+    const bool paged = page_table != nullptr;
+    if (!paged && params->cu_seqlens_k && !io->cu_seqlens_k_host) return FP2_ERR_INVALID_ARG;
     const int32_t* cu = io->cu_seqlens_host;
-    std::vector<int> q0(S), Lq(S), off(S);
+    const int32_t* cuk = io->cu_seqlens_k_host ? io->cu_seqlens_k_host : cu;
+    std::vector<int> q0(S), Lq(S), Lk(S), k0(S), off(S), pb(S);
     for (int b = 0; b < S; ++b) {
         q0[b] = cu[b];
         Lq[b] = cu[b + 1] - cu[b];
-        const int Lk = io->seqlens_k_host ? io->seqlens_k_host[b] : Lq[b];
-        if (q0[b] < 0 || Lq[b] < 0 || Lq[b] > kp.max_seqlen_q || Lk < Lq[b] ||
-            Lk > kp.max_seqlen_k || q0[b] + Lq[b] > kp.total_q)
+        Lk[b] = io->seqlens_k_host ? io->seqlens_k_host[b] : Lq[b];
+        k0[b] = paged ? 0 : cuk[b];
+        if (q0[b] < 0 || Lq[b] < 0 || Lq[b] > kp.max_seqlen_q || Lk[b] < Lq[b] ||
+            Lk[b] > kp.max_seqlen_k || q0[b] + Lq[b] > kp.total_q ||
+            (!paged && (k0[b] < 0 || k0[b] + Lk[b] > kp.total_k)))
             return FP2_ERR_INVALID_ARG;
-        off[b] = (Lk - Lq[b]) % block;
+        off[b] = (Lk[b] - Lq[b]) % block;
+        pb[b] = (Lk[b] - Lq[b]) / block;
     }
     const size_t elt_in = kp.fp8 ? 1 : 2, elt_out = kp.out_fp8 ? 1 : 2;
     const size_t row_in = (size_t)kp.Hq * kp.d * elt_in, row_out = (size_t)kp.Hq * kp.d * elt_out;
-    const size_t kv_bytes = (page_table ? (size_t)kp.num_pages * kp.page_size : (size_t)kp.total_k) *
-                            kp.Hkv * kp.d * elt_in;
+    const size_t row_kv = (size_t)kp.Hkv * kp.d * elt_in;
+    const size_t op_bytes = (size_t)S * kp.Hkv * kp.nkb_max * kp.d * elt_in;  // kbar_op / vbar_op
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP2_ERR_CUDA;
@@ -465,36 +473,70 @@ fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
     cudaStream_t down = io->download_stream ? static_cast<cudaStream_t>(io->download_stream) : s;
     auto* qh = static_cast<const uint8_t*>(io->q_host);
     auto* qd = static_cast<uint8_t*>(io->q_dev);
+    auto* kh = static_cast<const uint8_t*>(io->k_host);
+    auto* kd = static_cast<uint8_t*>(io->k_dev);
+    auto* vh = static_cast<const uint8_t*>(io->v_host);
+    auto* vd = static_cast<uint8_t*>(io->v_dev);
     auto* oh = static_cast<uint8_t*>(io->out_host);
     auto* od = static_cast<const uint8_t*>(io->out_dev);
+    auto h2d = [&](uint8_t* dst, const uint8_t* src, size_t at, size_t bytes) {
+        return cudaMemcpyAsync(dst + at, src + at, bytes, cudaMemcpyHostToDevice, up);
+    };
 
-    // K and V whole (any key block may be kept or averaged), then the means
+    // uploads start after the work already queued on params->stream
     cudaError_t e = join(s, up, ev[0]);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(io->k_dev, io->k_host, kv_bytes, cudaMemcpyHostToDevice, up);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(io->v_dev, io->v_host, kv_bytes, cudaMemcpyHostToDevice, up);
-    if (e == cudaSuccess) e = join(up, s, ev[1]);
-    if (e == cudaSuccess) e = fp2::launch_blockmean(kp, io->k_dev, io->v_dev, s);
-    // query-block ranges, highest (longest rows) first
+    int kb_done = 0;  // key blocks averaged so far
+    if (paged) {
+        // pages can sit anywhere in the cache: upload it whole, average every block
+        const size_t kv_bytes = (size_t)kp.num_pages * kp.page_size * row_kv;
+        if (e == cudaSuccess) e = h2d(kd, kh, 0, kv_bytes);
+        if (e == cudaSuccess) e = h2d(vd, vh, 0, kv_bytes);
+        if (e == cudaSuccess) e = join(up, s, ev[1]);
+        if (e == cudaSuccess) e = fp2::launch_blockmean(kp, kd, vd, s);
+        kb_done = kp.nkb_max;
+    } else {
+        // the mean tiles a range reads may reach blocks not averaged yet:
+        // zeros there (weight-0 columns of PV must meet finite values)
+        if (e == cudaSuccess) e = cudaMemsetAsync(kp.kbar_op, 0, op_bytes, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(kp.vbar_op, 0, op_bytes, s);
+    }
+    // query-block ranges, lowest first: a range needs the keys up to its last
+    // diagonal block, so the key upload grows with the ranges
     const int per = (kp.nqb_max + io->num_chunks - 1) / io->num_chunks;
     for (int c = 0; e == cudaSuccess && c < io->num_chunks; ++c) {
-        const int hi = kp.nqb_max - c * per, lo = std::max(0, hi - per);
-        if (hi <= 0) break;
+        const int lo = c * per, hi = std::min(kp.nqb_max, lo + per);
+        if (lo >= hi) break;
+        int kb_hi = kb_done;
+        if (!paged) {
+            for (int b = 0; b < S; ++b) kb_hi = std::max(kb_hi, pb[b] + hi);
+            kb_hi = std::min(kb_hi, kp.nkb_max);
+            for (int b = 0; e == cudaSuccess && b < S; ++b) {
+                const int r0 = kb_done * block, r1 = std::min(Lk[b], kb_hi * block);
+                if (r1 <= r0) continue;
+                const size_t at = (size_t)(k0[b] + r0) * row_kv, bytes = (size_t)(r1 - r0) * row_kv;
+                e = h2d(kd, kh, at, bytes);
+                if (e == cudaSuccess) e = h2d(vd, vh, at, bytes);
+            }
+        }
         // the sequences' query rows of blocks [lo, hi): rows t with
         // lo <= (off + t) / B < hi
         for (int b = 0; e == cudaSuccess && b < S; ++b) {
             const int r0 = std::max(0, lo * block - off[b]);
             const int r1 = std::min(Lq[b], hi * block - off[b]);
-            if (r1 > r0)
-                e = cudaMemcpyAsync(qd + (size_t)(q0[b] + r0) * row_in, qh + (size_t)(q0[b] + r0) * row_in,
-                                    (size_t)(r1 - r0) * row_in, cudaMemcpyHostToDevice, up);
+            if (r1 > r0) e = h2d(qd, qh, (size_t)(q0[b] + r0) * row_in, (size_t)(r1 - r0) * row_in);
         }
         if (e == cudaSuccess) e = join(up, s, ev[2 + 2 * c]);
+        if (e == cudaSuccess && kb_hi > kb_done) {
+            kp.kb_lo = kb_done;
+            kp.kb_n = kb_hi - kb_done;
+            e = fp2::launch_blockmean(kp, kd, vd, s);
+            kb_done = kb_hi;
+        }
         kp.qb_lo = lo;
         kp.qb_n = hi - lo;
-        if (e == cudaSuccess) e = fp2::launch_score(kp, io->q_dev, s);
+        if (e == cudaSuccess) e = fp2::launch_score(kp, qd, s);
         if (e == cudaSuccess) e = fp2::launch_mask(kp, tau, s);
-        if (e == cudaSuccess)
-            e = fp2::launch_attn(kp, io->q_dev, io->k_dev, io->v_dev, kp.kept_bits, io->out_dev, s);
+        if (e == cudaSuccess) e = fp2::launch_attn(kp, qd, kd, vd, kp.kept_bits, io->out_dev, s);
         if (e == cudaSuccess) e = join(s, down, ev[3 + 2 * c]);
         for (int b = 0; e == cudaSuccess && b < S; ++b) {
             const int r0 = std::max(0, lo * block - off[b]);
@@ -503,6 +545,12 @@ fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
                 e = cudaMemcpyAsync(oh + (size_t)(q0[b] + r0) * row_out, od + (size_t)(q0[b] + r0) * row_out,
                                     (size_t)(r1 - r0) * row_out, cudaMemcpyDeviceToHost, down);
         }
+    }
+    // blocks past every sequence's end get their zero means, as in fp2_prefill
+    if (e == cudaSuccess && kb_done < kp.nkb_max) {
+        kp.kb_lo = kb_done;
+        kp.kb_n = kp.nkb_max - kb_done;
+        e = fp2::launch_blockmean(kp, kd, vd, s);
     }
     // params->stream ends after the last download
     if (e == cudaSuccess) e = join(down, s, ev[kHostEvents - 1]);

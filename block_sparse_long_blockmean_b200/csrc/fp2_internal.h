@@ -18,6 +18,9 @@ struct KParams {
     // query blocks [qb_lo, qb_lo + qb_n) of every sequence are processed by
     // the score, mask and attention launches (all of them: 0, nqb_max)
     int qb_lo, qb_n;
+    // key blocks [kb_lo, kb_lo + kb_n) are averaged by the block-mean launch
+    // (all of them: 0, nkb_max)
+    int kb_lo, kb_n;
     int fp8;
     int uses_kv;               // 0: the launch never reads K/V (no key-extent check)
     int group_masks;           // score every head with its group's mean pooled query

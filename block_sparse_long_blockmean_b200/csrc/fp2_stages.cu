@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(128) blockmean_kernel(KParams p, const uint8_t
     constexpr int RPP = 128 / TPR;  // rows per pass
     __shared__ float red[2][RPP][D];
 
-    const int j = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int j = p.kb_lo + (int)blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
     const int nkb = (s.Lk + p.B - 1) / p.B;
@@ -346,7 +346,8 @@ __global__ void __launch_bounds__(128) mask_kernel(KParams p, float tau) {
 
 // -------------------------------------------------------------- launchers ---
 cudaError_t launch_blockmean(const KParams& p, const void* k, const void* v, cudaStream_t st) {
-    dim3 grid(p.nkb_max, p.Hkv, p.num_seqs);
+    dim3 grid(p.kb_n, p.Hkv, p.num_seqs);
+    if (p.kb_n <= 0) return cudaSuccess;
     auto K = static_cast<const uint8_t*>(k);
     auto V = static_cast<const uint8_t*>(v);
     if (p.fp8) {

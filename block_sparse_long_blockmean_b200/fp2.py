@@ -95,6 +95,7 @@ class HostIO(ctypes.Structure):
         ("out_dev", ctypes.c_void_p),
         ("cu_seqlens_host", ctypes.c_void_p),
         ("seqlens_k_host", ctypes.c_void_p),
+        ("cu_seqlens_k_host", ctypes.c_void_p),
         ("upload_stream", ctypes.c_void_p),
         ("download_stream", ctypes.c_void_p),
         ("num_chunks", ctypes.c_int),
@@ -211,7 +212,7 @@ def prefill_host(io: HostIO, page_table, cu_seqlens, tau: float, block: int, dty
 
 def host_io(q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_dev, cu_seqlens_host,
             seqlens_k_host=None, upload_stream=None, download_stream=None,
-            num_chunks: int = 8) -> HostIO:
+            num_chunks: int = 16, cu_seqlens_k_host=None) -> HostIO:
     """An ``fp2_host_io`` from tensors (host ones on the CPU, ideally pinned;
     int32 length arrays on the CPU) and torch streams (or None)."""
     io = HostIO()
@@ -220,6 +221,7 @@ def host_io(q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_dev, cu_s
     io.q_dev, io.k_dev, io.v_dev, io.out_dev = _ptr(q_dev), _ptr(k_dev), _ptr(v_dev), _ptr(out_dev)
     io.cu_seqlens_host = _ptr(cu_seqlens_host)
     io.seqlens_k_host = _ptr(seqlens_k_host)
+    io.cu_seqlens_k_host = _ptr(cu_seqlens_k_host)
     io.upload_stream = upload_stream.cuda_stream if upload_stream is not None else None
     io.download_stream = download_stream.cuda_stream if download_stream is not None else None
     io.num_chunks = int(num_chunks)

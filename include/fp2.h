@@ -237,6 +237,8 @@ typedef struct fp2_host_io {
     const int32_t* cu_seqlens_host; /* host copy of cu_seqlens [num_seqs+1] */
     const int32_t* seqlens_k_host;  /* host copy of params->seqlens_k [num_seqs],
                                        NULL when params->seqlens_k is NULL */
+    const int32_t* cu_seqlens_k_host; /* host copy of params->cu_seqlens_k [num_seqs+1],
+                                       NULL when that is NULL (contiguous K/V only) */
     void* upload_stream;   /* cudaStream_t for the host->device copies; NULL:
                               params->stream (no overlap) */
     void* download_stream; /* cudaStream_t for the device->host copies; NULL:
@@ -246,20 +248,20 @@ typedef struct fp2_host_io {
 
 /* fp2_prefill with q, K/V and out in host memory: the call a serving process
  * makes when the layer's inputs are not yet on the GPU (packaging of the
- * same method, not a step of it).  It uploads K and V and averages every
- * key block, then runs score, mask and attention over num_chunks ranges of
- * query blocks (highest first), uploading each range's query rows while the
- * previous range computes and downloading each range's output rows while
- * the next one computes.  Results are bit-identical to fp2_prefill on the
- * same data.
+ * same method, not a step of it).  It runs block means, score, mask and
+ * attention over num_chunks ranges of query blocks, lowest first, uploading
+ * each range's query rows (and, for contiguous K/V, the key blocks it adds)
+ * while the previous range computes, and downloading each range's output
+ * rows while the next one computes; a paged cache is uploaded whole first.
+ * Results are bit-identical to fp2_prefill on the same data.
  *  - Queues work on params->stream, io->upload_stream and
  *    io->download_stream and returns; params->stream is made to wait for the
  *    last download, so synchronising params->stream means out_host is done.
  *    The uploads first wait for work already queued on params->stream, so
  *    back-to-back calls on the same device buffers do not race.
- *  - cu_seqlens, params->seqlens_k and page_table stay device arrays (small,
- *    usually resident); cu_seqlens_host / seqlens_k_host must hold the same
- *    values (they place each range's query rows).
+ *  - cu_seqlens, params->seqlens_k, params->cu_seqlens_k and page_table
+ *    stay device arrays (small, usually resident); the *_host copies must
+ *    hold the same values (they place each range's rows).
  *  - Uses a library-owned pool of CUDA events per device, created on the
  *    first call (make it before any stream capture); calls from several
  *    host threads are serialised while they queue.

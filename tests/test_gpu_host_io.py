@@ -19,6 +19,8 @@ SHAPES = {
                             Hq=8, Hkv=2, page_size=64, dtype="fp8"),
     "chunk_g8_b64": dict(lens_q=[900, 5], lens_k=[900 + 333, 1000], Hq=16, Hkv=2, B=64,
                          page_size=32),
+    "mixed_contiguous": dict(lens_q=[1, 600, 0, 250, 1], lens_k=[2500, 600, 300, 1900, 129],
+                             Hq=8, Hkv=2),
 }
 
 
@@ -33,20 +35,25 @@ def device_reference(inp, tau, out_dtype=fp2.FP2_BF16):
 
 
 def host_call(pr, inp, tau, num_chunks, streams, out_host):
+    # the device buffers start as NaN bytes: every row the kernels read must
+    # have been uploaded by the call itself
+    for t in (pr.q, pr.k, pr.v, pr.out):
+        t.view(torch.uint8).fill_(0xFF)
     hq = inp.q.pin_memory()
     hk = inp.k.pin_memory()
     hv = inp.v.pin_memory()
     cu_h = inp.cu_seqlens_q.to(torch.int32).contiguous()
     lk_h = inp.seqlens_k.to(torch.int32).contiguous()
+    cuk_h = None if inp.paged else inp.cu_seqlens_k.to(torch.int32).contiguous()
     io = fp2.host_io(hq, hk, hv, out_host, pr.q, pr.k, pr.v, pr.out, cu_h, lk_h,
                      upload_stream=streams[0], download_stream=streams[1],
-                     num_chunks=num_chunks)
+                     num_chunks=num_chunks, cu_seqlens_k_host=cuk_h)
     fp2.prefill_host(io, pr.page_table, pr.cu_seqlens, tau, inp.shape.B, pr.dtype, pr.params)
-    return (hq, hk, hv, cu_h, lk_h)  # keep alive until the stream is synchronised
+    return (hq, hk, hv, cu_h, lk_h, cuk_h)  # keep alive until the stream is synchronised
 
 
 @pytest.mark.parametrize("name", sorted(SHAPES))
-@pytest.mark.parametrize("num_chunks", [1, 3, 8])
+@pytest.mark.parametrize("num_chunks", [1, 3, 16])
 def test_host_path_matches_device_path(name, num_chunks):
     inp = synth.make_inputs(H.small_shape(**SHAPES[name], seed=61))
     tau = H.pick_tau(H.oracle_scores(inp), 0.6)
