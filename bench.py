@@ -162,14 +162,20 @@ def algorithmic_flops(cnt, lens_q, lens_k, B, d):
     dropped = 0
     causal = 0
     for b, (Lq, Lk) in enumerate(zip(lens_q, lens_k)):
-        nqb = -(-Lq // B)
+        if Lq == 0:
+            continue
+        o = (Lk - Lq) % B                  # offset of the first query row in its block
+        nqb = -(-(o + Lq) // B)
         pb = (Lk - Lq) // B
         for i in range(nqb):
-            n_i = min(B, Lq - i * B)
+            r0, r1 = max(0, i * B - o), min(Lq, (i + 1) * B - o)
+            n_i = r1 - r0
             iabs = pb + i
+            # causal keys of the diagonal block, summed over the block's rows
+            diag = float(sum(range(r0 + o - i * B + 1, r1 + o - i * B + 1)))
             c = cnt[b, :, i].astype(np.float64)        # per head
             off = c - 1.0                               # kept off-diagonal blocks
-            kept_fl += float(off.sum()) * 4.0 * n_i * B * d + c.size * 2.0 * d * n_i * (n_i + 1)
+            kept_fl += float(off.sum()) * 4.0 * n_i * B * d + c.size * 4.0 * d * diag
             drop = (iabs + 1) - c
             corr_fl += float(drop.sum()) * 4.0 * d * n_i
             dropped += int(drop.sum())
@@ -382,7 +388,8 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
         "stage_ms": {"blockmean": stage_ms[0], "score": stage_ms[1], "mask": stage_ms[2],
                      "attn": stage_ms[3]},
         "kept_flops": kept_fl, "corr_flops": corr_fl, "clocks": clk, "dense": dense,
-        "union_inflation": union_ratio,
+        "union_inflation": union_ratio, "d": s.d,
+        "num_sms": torch.cuda.get_device_properties(dev).multi_processor_count,
         "e2e": e2e, "gen_s": gen_s, "inp": inp if want_cpu else None, "tau_inp": tau,
     }
     return res
@@ -532,6 +539,12 @@ def main():
 
     s_main, peak = summary(r)
     eff = s_main["eff_tflops_kept"]
+    # the second bound: exp2 per score on the MUFU unit, 16 per clock per SM
+    # (fp8 sends a quarter of them to the FMA pipe instead)
+    n_exp = (r["kept_flops"] + r["corr_flops"]) / (4.0 * r["d"])
+    sm_mhz = (r["clocks"] or {}).get("sm_mhz") or 1965.0
+    exp_peak = 16.0 * r["num_sms"] * sm_mhz * 1e6
+    exp_rate = n_exp / (r["stage_ms"]["attn"] * 1e-3)
     line = {
         "metric": METRIC, "value": ms_per_layer, "unit": "ms/layer", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -553,6 +566,10 @@ def main():
                      "kernel": "fp2_attn (attn_pair_kernel: G x block >= 256 packed rows)",
                      "peak_source": f"{peak_src} bf16_tflops_sustained" +
                                     (" x2 (fp8/bf16 nominal ratio)" if main_dt == "fp8" else "")},
+        "exp_roof": {"bound": "mufu", "achieved": exp_rate / 1e9, "peak": exp_peak / 1e9,
+                     "unit": "Gexp/s", "frac": exp_rate / exp_peak,
+                     "peak_source": f"16 ex2/clk/SM x {r['num_sms']} SMs x {sm_mhz:.0f} MHz "
+                                    "(median SM clock of the timed loop)"},
         "summary": {main_dt: s_main},
         "gpu_launches": 4 * args.steps,
         "clocks": r["clocks"],
