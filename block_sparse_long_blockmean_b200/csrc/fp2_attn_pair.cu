@@ -67,8 +67,10 @@ struct PairCfg {
 // K and V have separate rings: K(n) is free once QK_B(n) has run, V(n) only
 // after PV_B(n) -- a full MMA pair later -- so each stream refills as soon as
 // its own operand is consumed.
-enum { PB_K_FULL = 0, PB_K_EMPTY = 2, PB_V_FULL = 4, PB_V_EMPTY = 6, PB_Q_FULL = 8,
-       PB_S_FULL = 9, PB_P_READY = 11, PB_O_FINAL = 13, PB_DRAIN = 15, PB_COUNT = 16 };
+// KV_FULL[n % 2]: the producer's step n has landed, K(n) and V(n-1) together
+// (one barrier, so the MMA thread polls once per item for both)
+enum { PB_KV_FULL = 0, PB_K_EMPTY = 2, PB_V_EMPTY = 4, PB_Q_FULL = 6, PB_S_FULL = 7,
+       PB_P_READY = 9, PB_O_FINAL = 11, PB_DRAIN = 13, PB_COUNT = 14 };
 
 template <int D, int BLK, bool FP8>
 __global__ void __launch_bounds__(384, 1)
@@ -146,12 +148,15 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             prefetch_tmap(&maps.k);
             prefetch_tmap(&maps.v);
         }
-        // K runs one item ahead of V: iteration n loads K(n), then V(n-1)
-        int k_issued = 0, v_issued = 0;
+        // K runs one item ahead of V: step n loads K(n) and V(n-1), both
+        // counted on KV_FULL[n % 2] (K adds its bytes, V or a lone K arrives)
+        int steps = 0;  // 1 + the last producer step that issued a copy
         bool ok = true;
         for (int n = 0; n <= n_items; ++n) {
             if (n % 32 == 0 && n < n_items) fill_page_ring<BLK>(p, s, b, items, n_items, n, pring);
             if (lane == 0) {
+                uint64_t* full = &bars[PB_KV_FULL + n % C::S];
+                bool k_issued = false;
                 if (n < n_items) {
                     const int st = n % C::S;
                     if (n >= C::S && !mbar_wait(&bars[PB_K_EMPTY + st], ((n - C::S) / C::S) & 1,
@@ -161,9 +166,10 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                     } else {
                         issue_tile_load<D, BLK, FP8>(p, &maps.k, &maps.kb, s, b, hk, items[n],
                                                      pring + (n % kPageRing) * kMaxBoxes,
-                                                     sbase + C::OFF_K + st * C::KV_BYTES,
-                                                     &bars[PB_K_FULL + st], true);
-                        ++k_issued;
+                                                     sbase + C::OFF_K + st * C::KV_BYTES, full,
+                                                     n == 0);
+                        k_issued = true;
+                        steps = n + 1;
                     }
                 }
                 if (ok && n >= 1) {
@@ -172,24 +178,25 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                                                 abort_flag, kWaitLimitNs)) {
                         set_error(p.err, kErrTimeout, kDetWaitBase + 0);
                         ok = false;
+                        // K(n) went without an arrival: arrive so that the
+                        // step completes once its bytes land (drained below)
+                        if (k_issued) mbar_arrive(full);
                     } else {
                         issue_tile_load<D, BLK, FP8>(p, &maps.v, &maps.vb, s, b, hk, items[m],
                                                      pring + (m % kPageRing) * kMaxBoxes,
-                                                     sbase + C::OFF_V + st * C::KV_BYTES,
-                                                     &bars[PB_V_FULL + st], true);
-                        ++v_issued;
+                                                     sbase + C::OFF_V + st * C::KV_BYTES, full,
+                                                     true);
+                        steps = n + 1;
                     }
                 }
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         }
         if (lane == 0) {
-            // never leave with copies in flight
+            // never leave with copies in flight: the last steps that issued any
             volatile int no_abort = 0;
-            for (int n = max(0, k_issued - C::S); n < k_issued; ++n)
-                mbar_wait(&bars[PB_K_FULL + n % C::S], (n / C::S) & 1, &no_abort, kWaitLimitNs);
-            for (int n = max(0, v_issued - C::S); n < v_issued; ++n)
-                mbar_wait(&bars[PB_V_FULL + n % C::S], (n / C::S) & 1, &no_abort, kWaitLimitNs);
+            for (int n = max(0, steps - C::S); n < steps; ++n)
+                mbar_wait(&bars[PB_KV_FULL + n % C::S], (n / C::S) & 1, &no_abort, kWaitLimitNs);
             mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, kWaitLimitNs);
         }
       } else if (warp == 9 && lane == 0) {
@@ -202,14 +209,8 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             tc_fence_after();
             for (int n = 0; ok && n <= n_items; ++n) {
                 const int st = n & 1;
-                if (n < n_items &&
-                    !mbar_wait(&bars[PB_K_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs)) {
-                    set_error(p.err, kErrTimeout, kDetWaitBase + 2);
-                    ok = false;
-                    break;
-                }
-                if (n >= 1 && !mbar_wait(&bars[PB_V_FULL + ((n - 1) & 1)], ((n - 1) >> 1) & 1,
-                                         abort_flag, kWaitLimitNs)) {
+                // K(n) and V(n-1)
+                if (!mbar_wait(&bars[PB_KV_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs)) {
                     set_error(p.err, kErrTimeout, kDetWaitBase + 2);
                     ok = false;
                     break;
@@ -413,7 +414,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             if (X == 0 && item >= 0 && item * BLK + BLK > s.Lk) {
                 // V(n) loads one step behind K(n): let it land before zeroing
                 // (V(n+2) cannot reuse the slot before this warpgroup's P(n))
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[PB_V_FULL + (n & 1)], (n >> 1) & 1,
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[PB_KV_FULL + ((n + 1) & 1)], ((n + 1) >> 1) & 1,
                                                        abort_flag, kWaitLimitNs))) {
                     set_error(p.err, kErrTimeout, kDetWaitBase + 7);
                     ok = false;
