@@ -560,7 +560,7 @@ cudaError_t launch_attn_pair(const KParams& p, const void* q, const void* k, con
 // two-tile kernel; smaller ones to the single-tile kernel above.
 cudaError_t launch_attn(const KParams& p, const void* q, const void* k, const void* v,
                         const uint32_t* kept_bits, void* out, cudaStream_t st) {
-    if (p.G * p.B >= 256 && !getenv("FP2_SINGLE_TILE"))
+    if (!getenv("FP2_SINGLE_TILE"))
         return launch_attn_pair(p, q, k, v, kept_bits, out, st);
     if (p.fp8) {
         if (p.d == 128 && p.B == 128) return launch_attn_t<128, 128, true>(p, q, k, v, kept_bits, out, st);

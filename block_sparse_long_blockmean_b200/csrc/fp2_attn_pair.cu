@@ -1,6 +1,5 @@
-// fp2_attn_pair.cu -- the block-sparse attention kernel for query blocks of
-// at least 256 packed rows (G * block >= 256): two 128-row tiles per CTA
-// share every K/V tile and alternate on the tensor core.
+// fp2_attn_pair.cu -- the block-sparse attention kernel: two 128-row tiles
+// per CTA share every K/V tile and alternate on the tensor core.
 //
 // Same result as the single-tile kernel (fp2_attn.cu): for each query row an
 // online softmax over the tokens of the kept key blocks plus one pseudo-token
@@ -12,6 +11,11 @@
 // tokens [t0, t0+TOK) x G heads, tile B the next TOK tokens (TOK = 128/G).
 // Both tiles belong to query block i, so they walk the same list of kept
 // blocks and mean tiles, and each K/V tile is loaded once for 256 rows.
+// When a query block packs only 128 rows (G x block = 128: G = 1 with block
+// 128, G = 2 with block 64) tile A is query block i and tile B block i+1 of
+// the same KV head; the CTA walks the union of the two blocks' lists, and
+// each tile masks what its own block does not keep (tile A's rows take
+// nothing from block i+1, its causal future).
 //
 // Roles (384 threads = 3 warpgroups; registers rebalanced with setmaxnreg:
 // 224 per softmax thread, 56 in the control warpgroup, 384 x 168 in total):
@@ -91,22 +95,35 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     const int G = p.G;
     const int TOK = 128 / G;
+    // Tiles of one query block (G x block >= 256 packed rows: npair pairs of
+    // tiles per block), or, when a block is a single tile (G x block = 128),
+    // two adjacent query blocks i, i+1 (xq): they walk the union of their
+    // kept lists; a key block only the second keeps is masked out for the first.
     const int npair = BLK / (2 * TOK);
-    const int per_i = p.num_seqs * p.Hkv * npair;
-    const int i = p.qb_lo + p.qb_n - 1 - (int)(blockIdx.x / per_i);  // longest first
-    const int rem = (int)(blockIdx.x % per_i);
-    const int b = rem / (p.Hkv * npair);
-    const int hk = (rem / npair) % p.Hkv;
-    const int pr = rem % npair;
+    const bool xq = npair == 0;
+    const int units = xq ? (p.qb_n + 1) / 2 : p.qb_n;
+    const int per_u = p.num_seqs * p.Hkv * (xq ? 1 : npair);
+    const int u = units - 1 - (int)(blockIdx.x / per_u);  // longest first
+    const int rem = (int)(blockIdx.x % per_u);
+    const int b = rem / (p.Hkv * (xq ? 1 : npair));
+    const int hk = xq ? rem % p.Hkv : (rem / npair) % p.Hkv;
+    const int pr = xq ? 0 : rem % npair;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
-    // the pair's first query (negative inside a partial first query block)
-    const int t_begin = i * BLK - s.off + pr * 2 * TOK;
-    if (i >= s.nqb || t_begin >= s.Lq || t_begin + 2 * TOK <= 0) return;  // no rows here
+    const int i = p.qb_lo + (xq ? 2 * u : u);  // query block of tile A
+    const int i_b = xq ? i + 1 : i;            // query block of tile B
+    // whether tile B has rows (xq: block i+1 exists and is in this launch)
+    const bool b_ok = !xq || (i_b < s.nqb && i_b < p.qb_lo + p.qb_n);
+    // the tiles' first queries (negative inside a partial first query block)
+    const int t_a = i * BLK - s.off + pr * 2 * TOK;
+    const int t_b = xq ? i_b * BLK - s.off : t_a + TOK;
+    if (i >= s.nqb || t_a >= s.Lq || t_a + 2 * TOK <= 0) return;  // no rows here
     const int iabs = s.pb + i;
-    const int nw_c = (iabs + 32) / 32;
+    const int iabs_b = s.pb + i_b;
+    const int iabs_hi = b_ok ? iabs_b : iabs;  // last key block either tile reaches
+    const int nw_c = (iabs_hi + 32) / 32;
 
     if (threadIdx.x == 0) {
         for (int k = 0; k < PB_COUNT; ++k)
@@ -119,16 +136,18 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         for (int x = 0; x < 2; ++x)
             for (int c = 0; c < C::NCH; ++c)
                 tma_load_3d(q_s + x * C::Q_BYTES + c * (128 * 128), &maps.q, &bars[PB_Q_FULL],
-                            c * C::CH, hk * G, s.q0 + t_begin + x * TOK);
+                            c * C::CH, hk * G, s.q0 + (x ? t_b : t_a));
     }
     if (warp == 9) {
         tmem_alloc(&misc[0], 512);
         tmem_relinquish();
     }
+    // kept bits: G rows for tile A's block, then (xq) G rows for tile B's
     load_kept_bits(p, kept_bits, b, hk, i, iabs, nw_c, sbits);
+    if (xq && b_ok) load_kept_bits(p, kept_bits, b, hk, i_b, iabs_b, nw_c, sbits + G * nw_c);
     __syncthreads();
     if (warp == 8) {
-        const int n = build_items<BLK>(G, iabs, nw_c, sbits, items);
+        const int n = build_items<BLK>(xq && b_ok ? 2 * G : G, iabs_hi, nw_c, sbits, items);
         if (lane == 0) misc[2] = (uint32_t)n;
     }
     tc_fence_before();
@@ -269,14 +288,15 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         const int qw = warp & 3;
         const int r = qw * 32 + lane;             // row of the tile == TMEM lane
         const int g = r % G;
-        const int t = t_begin + X * TOK + r / G;  // query index in the sequence
+        const int t = (X ? t_b : t_a) + r / G;  // query index in the sequence
+        const int iabs_x = X && xq ? iabs_b : iabs;  // this tile's diagonal block
         const int h = hk * G + g;
-        const bool row_ok = t >= 0 && t < s.Lq;
+        const bool row_ok = t >= 0 && t < s.Lq && (X == 0 || b_ok);
         const int ppos = s.P + t;
         const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + X * 128;
         const uint32_t o_addr = tmem + lane_off + 256 + X * 128;
-        const uint32_t* hb = sbits + g * nw_c;
+        const uint32_t* hb = sbits + ((X && xq ? G : 0) + g) * nw_c;
         float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
         if constexpr (FP8) sl2 *= p.q_scale[h] * p.k_scale[hk];
         const float lb = __log2f((float)BLK);
@@ -303,9 +323,9 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 for (int w = 0; w < BLK / 32; ++w) {
                     const int j0 = tv * BLK + w * 32;
                     uint32_t dm = 0u;
-                    if (row_ok && j0 < iabs) {
+                    if (row_ok && j0 < iabs_x) {
                         dm = ~hb[j0 >> 5];
-                        const int nvalid = iabs - j0;
+                        const int nvalid = iabs_x - j0;
                         if (nvalid < 32) dm &= (1u << nvalid) - 1u;
                     }
                     dropped[w] = dm;
@@ -326,7 +346,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             tmem_wait_ld();
 
             if (item >= 0) {
-                if (live && item == iabs) {
+                if (live && item == iabs_x) {
                     const int lim = ppos - item * BLK;
 #pragma unroll
                     for (int c = 0; c < BLK; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
@@ -502,14 +522,17 @@ cudaError_t launch_attn_pair_t(const KParams& p, const void* q, const void* k, c
     if (!make_attn_maps(p, q, k, v, D, BLK, TOK, &maps)) return cudaErrorInvalidValue;
     const int items_cap = p.nkb_max + (p.nkb_max + BLK - 1) / BLK + 2;
     const int nw_c_max = p.nkb_max / 32 + 1;
-    size_t smem = 1024 + C::OFF_ITEMS + (size_t)items_cap * 4 + (size_t)p.G * nw_c_max * 4;
+    const bool xq = BLK < 2 * TOK;  // tiles are adjacent query blocks: twice the kept bits
+    size_t smem = 1024 + C::OFF_ITEMS + (size_t)items_cap * 4 +
+                  (size_t)(xq ? 2 : 1) * p.G * nw_c_max * 4;
     if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM: it owns all 512 TMEM columns
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attn_pair_kernel<D, BLK, FP8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int npair = BLK / (2 * TOK);
-    const long long grid = (long long)p.qb_n * p.num_seqs * p.Hkv * npair;
+    const long long grid = xq ? (long long)((p.qb_n + 1) / 2) * p.num_seqs * p.Hkv
+                              : (long long)p.qb_n * p.num_seqs * p.Hkv * npair;
     if (grid <= 0) return cudaSuccess;
     attn_pair_kernel<D, BLK, FP8><<<(unsigned)grid, 384, smem, st>>>(
         p, maps, kept_bits, static_cast<__nv_bfloat16*>(out), items_cap);

@@ -48,9 +48,10 @@
  *    G = Hq/Hkv in {1,2,4,8} with 128/G <= block, page_size a power of two
  *    in [16, 256] that divides the block or is divided by it.
  *
- * Kernel choice: problems with G * block >= 256 packed rows per query block
- * run the two-tile attention kernel, smaller ones the one-tile kernel; the
- * environment variable FP2_SINGLE_TILE=1 forces the one-tile kernel (tests).
+ * Kernel choice: the two-tile attention kernel runs every problem (two
+ * 128-row tiles of one query block when G * block >= 256, else two adjacent
+ * query blocks); the environment variable FP2_SINGLE_TILE=1 forces the
+ * one-tile kernel instead (tests).
  *
  * Errors: argument errors are returned synchronously before any launch.
  * CUDA launch errors return FP2_ERR_CUDA.  Problems only the device can see
