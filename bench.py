@@ -563,7 +563,7 @@ def main():
                    "output": "e4m3 for the fp8 run" if args.out_fp8 else "bf16"},
         "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
                      "frac": eff / peak, "traffic": recorded_traffic(main_dt),
-                     "kernel": "fp2_attn (attn_pair_kernel: G x block >= 256 packed rows)",
+                     "kernel": "fp2_attn (attn_pair_kernel)",
                      "peak_source": f"{peak_src} bf16_tflops_sustained" +
                                     (" x2 (fp8/bf16 nominal ratio)" if main_dt == "fp8" else "")},
         "exp_roof": {"bound": "mufu", "achieved": exp_rate / 1e9, "peak": exp_peak / 1e9,
