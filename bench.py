@@ -483,6 +483,21 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+def job_time(local_ms: float, steps: int, world: int):
+    """(timed region of the job, whole-job ms per layer): the slowest rank's
+    device time (all-reduce MAX over the process group, gloo or nccl), and
+    that time over the layers all ranks processed, one per rank per step."""
+    total = float(local_ms)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    return total, total / (steps * world)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -507,12 +522,7 @@ def main():
         results[dn] = run_gpu(args, rank, world, dn, want_cpu=(dn == dtypes[0]))
     main_dt = dtypes[0]
     r = results[main_dt]
-    total_ms = r["total_ms"]
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
-    ms_per_layer = total_ms / (args.steps * world)
+    total_ms, ms_per_layer = job_time(r["total_ms"], args.steps, world)
 
     def summary(x):
         attn_ms = x["stage_ms"]["attn"]
