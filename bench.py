@@ -555,24 +555,29 @@ def main():
     sm_mhz = (r["clocks"] or {}).get("sm_mhz") or 1965.0
     exp_peak = 16.0 * r["num_sms"] * sm_mhz * 1e6
     exp_rate = n_exp / (r["stage_ms"]["attn"] * 1e-3)
+    wl = synth.workload(args.workload)
+    in_bytes = (sum(wl.lens_q) * wl.Hq + 2 * sum(wl.lens_k) * wl.Hkv) * wl.d * \
+        (1 if main_dt == "fp8" else 2)
     line = {
         "metric": METRIC, "value": ms_per_layer, "unit": "ms/layer", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": main_dt,
         "data": "synthetic",
         "config": {"workload": synth.WORKLOAD_NAMES[args.workload],
-                   "seq_len": synth.workload(args.workload).lens_q[0],
-                   "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128, "block": 128,
-                   "target_drop": args.drop if args.drop is not None else
-                   synth.workload(args.workload).drop,
-                   "layout": "paged K/V (64-token pages)" if synth.workload(args.workload).page_size
+                   "seq_len": wl.lens_q[0], "prefix_len": wl.lens_k[0] - wl.lens_q[0],
+                   "num_q_heads": wl.Hq, "num_kv_heads": wl.Hkv, "head_dim": wl.d,
+                   "block": wl.B,
+                   "target_drop": args.drop if args.drop is not None else wl.drop,
+                   "layout": f"paged K/V ({wl.page_size}-token pages)" if wl.page_size
                    else "contiguous K/V",
-                   "l2": "inputs (1.6 GB) larger than L2; no flush",
+                   "l2": f"inputs ({in_bytes / 1e9:.2f} GB) larger than L2; no flush",
                    "per_gpu": "one independent layer per GPU",
                    "masks": "per KV group (variant)" if args.group_masks else "per query head",
                    "output": "e4m3 for the fp8 run" if args.out_fp8 else "bf16"},
         "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
-                     "frac": eff / peak, "traffic": recorded_traffic(main_dt),
+                     "frac": eff / peak,
+                     # the ncu figure is for the 128K layer's launch only
+                     "traffic": recorded_traffic(main_dt) if args.workload == WORKLOAD_ID else None,
                      "kernel": "fp2_attn (attn_pair_kernel)",
                      "peak_source": f"{peak_src} bf16_tflops_sustained" +
                                     (" x2 (fp8/bf16 nominal ratio)" if main_dt == "fp8" else "")},
