@@ -18,6 +18,9 @@ CASES = {
     "varlen_paged_g8_fp8": dict(lens_q=[700, 300], lens_k=[1024 + 700, 300], Hq=16, Hkv=2,
                                 page_size=64, dtype="fp8"),
     "tiny_g4_d64_b64": dict(lens_q=[1024], Hq=4, Hkv=1, d=64, B=64, latents="per_block"),
+    # G x block = 128: the two tiles of a CTA are adjacent query blocks
+    "g2_b64_pairs_of_blocks": dict(lens_q=[1000, 1], lens_k=[1000, 777], Hq=4, Hkv=2, B=64),
+    "g1_mha_unaligned": dict(lens_q=[300, 90], lens_k=[300 + 61, 90], Hq=4, Hkv=4),
 }
 
 
