@@ -21,7 +21,8 @@
 // 224 per softmax thread, 56 in the control warpgroup, 384 x 168 in total):
 //   warps 0-3  softmax for tile A (thread = row = TMEM lane)
 //   warps 4-7  softmax for tile B
-//   warp 8     TMA producer (both Q tiles, then the K/V ring of 2 stages)
+//   warp 8     TMA producer of the K and V rings (2 stages each; the two Q
+//              tiles are fetched by thread 0 right after the barriers exist)
 //   warps 10-11 idle
 //   warp 9     TMEM owner; lane 0 issues the MMAs in the order
 //                PV_A(n-1), QK_A(n), PV_B(n-1), QK_B(n)
