@@ -1,0 +1,53 @@
+"""bench.py's useful-work count (the numerator of its TFLOP/s and roofline)
+against brute force over the oracle's masks: 4*d flops for every (query row,
+kept key token at or before the row) pair, and 4*d for every (query row,
+dropped block) pseudo-token, on prefixes aligned and not."""
+import math
+
+import numpy as np
+import pytest
+
+import bench
+from oracle import oracle as O
+
+
+def brute(keeps, lens_q, lens_k, B, d, Hq):
+    kept = corr = 0
+    for b, (Lq, Lk) in enumerate(zip(lens_q, lens_k)):
+        P = Lk - Lq
+        for t in range(Lq):
+            p = P + t
+            iabs = p // B
+            i = iabs - P // B
+            for h in range(Hq):
+                for j in range(iabs + 1):
+                    if keeps[b][h, i, j]:
+                        kept += min(p, (j + 1) * B - 1) - j * B + 1
+                    else:
+                        corr += 1
+    return 4.0 * d * kept, 4.0 * d * corr
+
+
+@pytest.mark.parametrize("lens_q,lens_k,B", [
+    ([200], [200], 32),
+    ([37, 1, 90], [100, 61, 90], 16),       # prefixes 63 and 60: unaligned, a decode row
+    ([64, 50], [64 + 32, 50 + 48], 32),     # aligned prefixes
+])
+def test_flop_count_matches_brute_force(lens_q, lens_k, B):
+    rng = np.random.default_rng(17)
+    Hq, Hkv, d = 4, 2, 8
+    keeps = []
+    nqb_max = max(-(-((Lk - Lq) % B + Lq) // B) for Lq, Lk in zip(lens_q, lens_k))
+    cnt = np.zeros((len(lens_q), Hq, nqb_max), dtype=np.int32)
+    for b, (Lq, Lk) in enumerate(zip(lens_q, lens_k)):
+        Q = rng.standard_normal((Lq, Hq, d)) * 1.5
+        K = rng.standard_normal((Lk, Hkv, d)) * 1.5
+        V = rng.standard_normal((Lk, Hkv, d))
+        r = O.prefill_seq(Q, K, V, B, 0.4)
+        keeps.append(r.keep)
+        cnt[b, :, : r.keep.shape[1]] = r.keep.sum(axis=2)
+    kept, corr, drop = bench.algorithmic_flops(cnt, lens_q, lens_k, B, d)
+    want_kept, want_corr = brute(keeps, lens_q, lens_k, B, d, Hq)
+    assert kept == pytest.approx(want_kept, rel=0, abs=0.5)
+    assert corr == pytest.approx(want_corr, rel=0, abs=0.5)
+    assert 0.0 < drop < 1.0 and math.isfinite(drop)
