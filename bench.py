@@ -434,6 +434,24 @@ def cpu_baseline(inp, tau, budget_blocks=4, heads_per_block=8):
                        f"attention scaled x{scale:.0f}")}
 
 
+def run_config(args, dtype_name: str) -> dict:
+    """The workload description both arms print in their JSON line."""
+    from block_sparse_long_blockmean_b200 import synth
+    wl = synth.workload(args.workload)
+    in_bytes = (sum(wl.lens_q) * wl.Hq + 2 * sum(wl.lens_k) * wl.Hkv) * wl.d * \
+        (1 if dtype_name == "fp8" else 2)
+    return {"workload": synth.WORKLOAD_NAMES[args.workload],
+            "seq_len": wl.lens_q[0], "prefix_len": wl.lens_k[0] - wl.lens_q[0],
+            "num_q_heads": wl.Hq, "num_kv_heads": wl.Hkv, "head_dim": wl.d, "block": wl.B,
+            "target_drop": args.drop if args.drop is not None else wl.drop,
+            "layout": f"paged K/V ({wl.page_size}-token pages)" if wl.page_size
+            else "contiguous K/V",
+            "l2": f"inputs ({in_bytes / 1e9:.2f} GB) larger than L2; no flush",
+            "per_gpu": "one independent layer per GPU",
+            "masks": "per KV group (variant)" if args.group_masks else "per query head",
+            "output": "e4m3 for the fp8 run" if args.out_fp8 else "bf16"}
+
+
 def reference_arm(args):
     """--impl reference: the fp64 CPU oracle as it stands, each step a bounded
     sample of the same layer (one query block x 4 heads), scaled to ms/layer."""
@@ -444,6 +462,7 @@ def reference_arm(args):
     s = shape
     B = s.B
     K, V = inp.seq_k(0), inp.seq_v(0)
+    t_sel = time.time()
     kbar, vbar, cnt = O.blockmean(K, V, B)
     Lq = s.lens_q[0]
     nqb = -(-Lq // B)
@@ -451,8 +470,11 @@ def reference_arm(args):
     for i0 in range(0, nqb, 64):
         parts.append(O.pool_q(inp._deq(inp.q[i0 * B: (i0 + 64) * B], None), B))
     S = O.score(np.concatenate(parts, axis=1), kbar, 0)
+    t_sel = time.time() - t_sel  # block means, pooled scores of the whole layer
     tau = O.tau_for_drop([S], [0], args.drop if args.drop is not None else shape.drop)
+    t_m = time.time()
     keep = O.mask(S, 0, tau)
+    t_sel += time.time() - t_m
     rng = np.random.default_rng(0)
     times = []
     heads = np.arange(4, dtype=np.int32)
@@ -466,18 +488,19 @@ def reference_arm(args):
         # the cost of a block grows with its kept blocks; scale to the layer
         kept_i = keep[:4, i].sum()
         if it >= args.warmup:
-            times.append(dt * kept_all / max(kept_i, 1))
+            times.append(t_sel + dt * kept_all / max(kept_i, 1))
     ms = float(np.mean(times)) * 1e3
     line = {"metric": METRIC, "value": ms, "unit": "ms/layer", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": synth.WORKLOAD_NAMES[args.workload],
-                       "drop": args.drop if args.drop is not None else shape.drop},
+            "config": run_config(args, "bf16"),
             "cpu_baseline": {"value": ms, "unit": "ms/layer", "cores": O.num_threads(),
                              "kind": "oracle",
-                             "sample": "per step: corrected attention of 4 heads x 1 random "
-                                       "query block, scaled by kept-block count to the layer"},
+                             "sample": f"the whole layer's block means, pooled scores and mask "
+                                       f"({t_sel:.1f} s, once) + per step the corrected attention "
+                                       f"of 4 heads x 1 random query block, scaled by kept-block "
+                                       f"count to the layer"},
             "e2e": {"value": ms, "unit": "ms/layer", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -555,25 +578,12 @@ def main():
     sm_mhz = (r["clocks"] or {}).get("sm_mhz") or 1965.0
     exp_peak = 16.0 * r["num_sms"] * sm_mhz * 1e6
     exp_rate = n_exp / (r["stage_ms"]["attn"] * 1e-3)
-    wl = synth.workload(args.workload)
-    in_bytes = (sum(wl.lens_q) * wl.Hq + 2 * sum(wl.lens_k) * wl.Hkv) * wl.d * \
-        (1 if main_dt == "fp8" else 2)
     line = {
         "metric": METRIC, "value": ms_per_layer, "unit": "ms/layer", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": main_dt,
         "data": "synthetic",
-        "config": {"workload": synth.WORKLOAD_NAMES[args.workload],
-                   "seq_len": wl.lens_q[0], "prefix_len": wl.lens_k[0] - wl.lens_q[0],
-                   "num_q_heads": wl.Hq, "num_kv_heads": wl.Hkv, "head_dim": wl.d,
-                   "block": wl.B,
-                   "target_drop": args.drop if args.drop is not None else wl.drop,
-                   "layout": f"paged K/V ({wl.page_size}-token pages)" if wl.page_size
-                   else "contiguous K/V",
-                   "l2": f"inputs ({in_bytes / 1e9:.2f} GB) larger than L2; no flush",
-                   "per_gpu": "one independent layer per GPU",
-                   "masks": "per KV group (variant)" if args.group_masks else "per query head",
-                   "output": "e4m3 for the fp8 run" if args.out_fp8 else "bf16"},
+        "config": run_config(args, main_dt),
         "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
                      "frac": eff / peak,
                      # the ncu figure is for the 128K layer's launch only
