@@ -61,14 +61,19 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_pair_128k_traffic.md")
 
 
 def attn_source_hash() -> str:
-    """sha256 (12 hex) over the attention kernel's sources: ties a recorded ncu
-    traffic figure to the exact kernel it was taken on."""
+    """sha256 (12 hex) over the attention kernel's sources with comments and
+    whitespace removed: ties a recorded ncu traffic figure to the exact code
+    it was taken on (editing a comment does not change the kernel)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_long_blockmean_b200", "csrc")
     for f in ATTN_SOURCES:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f)) as fh:
+            code = fh.read()
+        code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
+        code = re.sub(r"//[^\n]*", " ", code)
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()[:12]
 
 

@@ -11,6 +11,10 @@
 //     logit q.kbar_j/sqrt(d) + ln(n_j) with n_j = B (dropped blocks are
 //     always full), value vbar_j.
 //
+// This one-tile kernel runs only when FP2_SINGLE_TILE is set (the two-tile
+// kernel of fp2_attn_pair.cu takes every problem otherwise); the tests keep
+// it as an independent second implementation of the same operator.
+//
 // Work item = (sequence, KV head, query block i, slice tq): 128 tensor-core
 // rows = 128/G query tokens x the G query heads of the KV head (PackGQA: the
 // K/V tile of a block is loaded once and used by all G heads).  The item
