@@ -39,9 +39,10 @@ def parse():
     ap.add_argument("--dtype", default="both", choices=["bf16", "fp8", "both"])
     ap.add_argument("--drop", type=float, default=None,
                     help="target dropped fraction (default: the workload's, 0.8 at 128K)")
-    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[2, 3, 5],
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=[2, 3, 4, 5],
                     help="3 = the 128K layer (the metric's workload); 2 = the 32K layer, a "
-                         "smaller case for profiler captures; 5 = a 32K chunk on a "
+                         "smaller case for profiler captures; 4 = 8 varlen sequences on a "
+                         "paged cache with permuted pages; 5 = a 32K chunk on a "
                          "229376-token paged prefix (also times the block-mean cache)")
     ap.add_argument("--out-fp8", action="store_true",
                     help="e4m3 output (fp8 runs; default scale: the KV head's v_scale)")
@@ -400,43 +401,84 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
     return res
 
 
-def cpu_baseline(inp, tau, budget_blocks=4, heads_per_block=8):
-    """The fp64 oracle on a bounded sample of the same layer: every block
-    mean, pooled score and mask of the whole layer, then the corrected
-    attention of `heads_per_block` heads x all rows of `budget_blocks` query
-    blocks at evenly spaced depths; the attention time is scaled to all
-    blocks and heads (its cost grows linearly with the block index)."""
+def oracle_seq_scores(inp, b):
+    """The oracle's block means, pooled queries and block scores of sequence
+    ``b``: (K, V, kbar, vbar, cnt, S, pb, off).  The queries are dequantised
+    and pooled 64 blocks at a time, so host memory stays bounded on long
+    sequences; a prefix that is not a multiple of B shortens the first block."""
     from oracle import oracle as O
     s = inp.shape
     B = s.B
-    t0 = time.time()
-    K, V = inp.seq_k(0), inp.seq_v(0)
+    K, V = inp.seq_k(b), inp.seq_v(b)
     kbar, vbar, cnt = O.blockmean(K, V, B)
-    Lq = s.lens_q[0]
-    pb = (s.lens_k[0] - Lq) // B
-    nqb = -(-Lq // B)
+    Lq, Lk = s.lens_q[b], s.lens_k[b]
+    pb, off = (Lk - Lq) // B, (Lk - Lq) % B
+    if Lq == 0:
+        return K, V, kbar, vbar, cnt, np.zeros((s.Hq, 0, kbar.shape[1])), pb, off
+    nqb = -(-(off + Lq) // B)
+    a = int(inp.cu_seqlens_q[b])
     parts = []
     for i0 in range(0, nqb, 64):
-        Qc = inp._deq(inp.q[i0 * B: min(Lq, (i0 + 64) * B)], inp.q_scale)
-        parts.append(O.pool_q(Qc, B))
-    qbar = np.concatenate(parts, axis=1)
-    S = O.score(qbar, kbar, pb)
-    keep = O.mask(S, pb, tau)
-    t_sel = time.time() - t0
-    blocks = [int((m + 0.5) * nqb / budget_blocks) for m in range(budget_blocks)]
+        r0, r1 = max(0, i0 * B - off), min(Lq, (i0 + 64) * B - off)
+        parts.append(O.pool_q(inp._deq(inp.q[a + r0: a + r1], inp.q_scale), B,
+                              off if i0 == 0 else 0))
+    S = O.score(np.concatenate(parts, axis=1), kbar, pb)
+    return K, V, kbar, vbar, cnt, S, pb, off
+
+
+def oracle_block(inp, b, i, seq, keep, heads):
+    """The oracle's corrected attention of query block ``i`` of sequence
+    ``b`` for ``heads`` (``seq`` = that sequence's oracle_seq_scores):
+    ``[rows * len(heads), d]`` ordered (row, head)."""
+    from oracle import oracle as O
+    K, V, kbar, vbar, cnt, _, pb, off = seq
+    B = inp.shape.B
+    r0, r1 = max(0, i * B - off), min(inp.shape.lens_q[b], (i + 1) * B - off)
+    a = int(inp.cu_seqlens_q[b])
+    Qb = inp._deq(inp.q[a + r0: a + r1], inp.q_scale)
+    return O.attn_query_block(Qb, K, V, kbar, vbar, cnt, keep[:, i], B, pb + i, heads,
+                              p0=(pb * B + off) + r0)
+
+
+def cpu_baseline(inp, tau, budget_blocks=4, heads_per_block=8):
+    """The fp64 oracle on a bounded sample of the same layer: every block
+    mean, pooled score and mask of every sequence, then the corrected
+    attention of `heads_per_block` heads x all rows of about `budget_blocks`
+    query blocks at evenly spaced depths (at least one per sequence).  Each
+    sequence's attention time is scaled to all its blocks and heads by kept
+    block pairs, which is what the oracle's attention cost grows with."""
+    from oracle import oracle as O
+    s = inp.shape
+    B = s.B
     heads = np.arange(heads_per_block, dtype=np.int32)
-    t1 = time.time()
-    for i in blocks:
-        Qb = inp._deq(inp.q[i * B: min(Lq, (i + 1) * B)], inp.q_scale)
-        O.attn_query_block(Qb, K, V, kbar, vbar, cnt, keep[:, i], B, pb + i, heads)
-    t_attn = time.time() - t1
-    scale = (nqb / budget_blocks) * (s.Hq / heads_per_block)
-    est_s = t_sel + t_attn * scale
+    nqb_all = [-(-((Lk - Lq) % B + Lq) // B) for Lq, Lk in zip(s.lens_q, s.lens_k)]
+    t_sel = t_attn = est_attn = 0.0
+    n_blocks = 0
+    for b in range(inp.num_seqs):
+        if s.lens_q[b] == 0:
+            continue
+        t0 = time.time()
+        seq = oracle_seq_scores(inp, b)
+        keep = O.mask(seq[5], seq[6], tau)
+        t_sel += time.time() - t0
+        nqb = nqb_all[b]
+        m = max(1, round(budget_blocks * nqb / sum(nqb_all)))
+        blocks = sorted({int((x + 0.5) * nqb / m) for x in range(m)})
+        t1 = time.time()
+        for i in blocks:
+            oracle_block(inp, b, i, seq, keep, heads)
+        dt = time.time() - t1
+        t_attn += dt
+        n_blocks += len(blocks)
+        sampled = int(keep[:heads_per_block][:, blocks].sum())
+        est_attn += dt * int(keep.sum()) / max(sampled, 1)
+        del seq, keep
+    est_s = t_sel + est_attn
     return {"value": est_s * 1e3, "unit": "ms/layer", "cores": O.num_threads(), "kind": "oracle",
-            "sample": (f"whole-layer block means, pooled scores and mask ({t_sel:.1f} s) + "
-                       f"corrected attention of {heads_per_block}/{s.Hq} heads x "
-                       f"{budget_blocks}/{nqb} query blocks ({t_attn:.1f} s), "
-                       f"attention scaled x{scale:.0f}")}
+            "sample": (f"block means, pooled scores and masks of all {inp.num_seqs} sequence(s) "
+                       f"({t_sel:.1f} s) + corrected attention of {heads_per_block}/{s.Hq} heads x "
+                       f"{n_blocks}/{sum(nqb_all)} query blocks ({t_attn:.1f} s), each "
+                       f"sequence's attention scaled by its kept block pairs")}
 
 
 def run_config(args, dtype_name: str) -> dict:
@@ -445,8 +487,12 @@ def run_config(args, dtype_name: str) -> dict:
     wl = synth.workload(args.workload)
     in_bytes = (sum(wl.lens_q) * wl.Hq + 2 * sum(wl.lens_k) * wl.Hkv) * wl.d * \
         (1 if dtype_name == "fp8" else 2)
-    return {"workload": synth.WORKLOAD_NAMES[args.workload],
-            "seq_len": wl.lens_q[0], "prefix_len": wl.lens_k[0] - wl.lens_q[0],
+    lens = {"seq_len": wl.lens_q[0], "prefix_len": wl.lens_k[0] - wl.lens_q[0]}
+    if len(wl.lens_q) > 1:
+        lens = {"global_batch": len(wl.lens_q), "seq_lens": list(wl.lens_q),
+                "prefix_lens": [k - q for q, k in zip(wl.lens_q, wl.lens_k)],
+                "total_tokens": int(sum(wl.lens_q))}
+    return {"workload": synth.WORKLOAD_NAMES[args.workload], **lens,
             "num_q_heads": wl.Hq, "num_kv_heads": wl.Hkv, "head_dim": wl.d, "block": wl.B,
             "target_drop": args.drop if args.drop is not None else wl.drop,
             "layout": f"paged K/V ({wl.page_size}-token pages)" if wl.page_size
@@ -458,42 +504,44 @@ def run_config(args, dtype_name: str) -> dict:
 
 
 def reference_arm(args):
-    """--impl reference: the fp64 CPU oracle as it stands, each step a bounded
-    sample of the same layer (one query block x 4 heads), scaled to ms/layer."""
+    """--impl reference: the fp64 CPU oracle as it stands.  Block means,
+    pooled scores and masks of every sequence are timed once; each step then
+    times the corrected attention of one random query block x 4 heads and
+    scales it to the layer by kept block pairs."""
     from block_sparse_long_blockmean_b200 import synth
     from oracle import oracle as O
     shape = synth.workload(args.workload, "bf16")
     inp = synth.make_inputs(shape)
     s = shape
-    B = s.B
-    K, V = inp.seq_k(0), inp.seq_v(0)
     t_sel = time.time()
-    kbar, vbar, cnt = O.blockmean(K, V, B)
-    Lq = s.lens_q[0]
-    nqb = -(-Lq // B)
-    parts = []
-    for i0 in range(0, nqb, 64):
-        parts.append(O.pool_q(inp._deq(inp.q[i0 * B: (i0 + 64) * B], None), B))
-    S = O.score(np.concatenate(parts, axis=1), kbar, 0)
-    t_sel = time.time() - t_sel  # block means, pooled scores of the whole layer
-    tau = O.tau_for_drop([S], [0], args.drop if args.drop is not None else shape.drop)
+    S_list, pb_list = [], []
+    for b in range(inp.num_seqs):
+        seq = oracle_seq_scores(inp, b)
+        S_list.append(seq[5])
+        pb_list.append(seq[6])
+        del seq
+    t_sel = time.time() - t_sel
+    tau = O.tau_for_drop(S_list, pb_list, args.drop if args.drop is not None else shape.drop)
     t_m = time.time()
-    keep = O.mask(S, 0, tau)
+    keeps = [O.mask(S, pb, tau) for S, pb in zip(S_list, pb_list)]
     t_sel += time.time() - t_m
+    del S_list
+    blocks = [(b, i) for b in range(inp.num_seqs) for i in range(keeps[b].shape[1])]
+    kept_all = sum(int(k.sum()) for k in keeps)
     rng = np.random.default_rng(0)
-    times = []
     heads = np.arange(4, dtype=np.int32)
-    kept_all = keep.sum()
+    cached = (None, None)
+    times = []
     for it in range(args.warmup + args.steps):
-        i = int(rng.integers(0, nqb))
-        Qb = inp._deq(inp.q[i * B: (i + 1) * B], None)
+        b, i = blocks[int(rng.integers(0, len(blocks)))]
+        if cached[0] != b:
+            # the sequence's K/V and block means (their time is in t_sel)
+            cached = (b, oracle_seq_scores(inp, b))
         t0 = time.time()
-        O.attn_query_block(Qb, K, V, kbar, vbar, cnt, keep[:, i], B, i, heads)
+        oracle_block(inp, b, i, cached[1], keeps[b], heads)
         dt = time.time() - t0
-        # the cost of a block grows with its kept blocks; scale to the layer
-        kept_i = keep[:4, i].sum()
         if it >= args.warmup:
-            times.append(t_sel + dt * kept_all / max(kept_i, 1))
+            times.append(t_sel + dt * kept_all / max(int(keeps[b][:4, i].sum()), 1))
     ms = float(np.mean(times)) * 1e3
     line = {"metric": METRIC, "value": ms, "unit": "ms/layer", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -502,10 +550,10 @@ def reference_arm(args):
             "config": run_config(args, "bf16"),
             "cpu_baseline": {"value": ms, "unit": "ms/layer", "cores": O.num_threads(),
                              "kind": "oracle",
-                             "sample": f"the whole layer's block means, pooled scores and mask "
-                                       f"({t_sel:.1f} s, once) + per step the corrected attention "
-                                       f"of 4 heads x 1 random query block, scaled by kept-block "
-                                       f"count to the layer"},
+                             "sample": f"block means, pooled scores and masks of all "
+                                       f"{inp.num_seqs} sequence(s) ({t_sel:.1f} s, once) + per "
+                                       f"step the corrected attention of 4 heads x 1 random query "
+                                       f"block, scaled by kept block pairs to the layer"},
             "e2e": {"value": ms, "unit": "ms/layer", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
