@@ -46,6 +46,19 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(fp2.SIGNATURES) == set(declared_functions())
 
 
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c99"), ("g++", "-std=c++11")])
+def test_header_is_strict_c99_and_cxx11(tmp_path, compiler, std):
+    """The boundary is plain C: the header compiles alone, warning-free, as
+    pedantic C99 and as C++11 (extern "C")."""
+    src = tmp_path / "hdr.c"
+    src.write_text('#include "fp2.h"\nint main(void) { return (int)sizeof(fp2_params) == 0; }\n')
+    cmd = [compiler, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+           os.path.join(ROOT, "include")]
+    if compiler == "g++":
+        cmd += ["-x", "c++"]
+    subprocess.run(cmd + [str(src), "-o", str(tmp_path / "hdr")], check=True)
+
+
 def test_struct_layout_matches_header(tmp_path):
     fields = [f for f, _ in fp2.Params._fields_]
     lfields = [f for f, _ in fp2.WorkspaceLayout._fields_]
