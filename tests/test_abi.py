@@ -110,6 +110,37 @@ def test_workspace_layout_for_the_128k_layer(lib):
     assert fp2.workspace_size(P, 128) == L.total
 
 
+@pytest.mark.parametrize("S,Hq,Hkv,d,max_q,max_k,B", [
+    (1, 4, 1, 64, 1024, 1024, 64),           # tiny causal layer
+    (3, 32, 8, 128, 1000, 5000, 128),        # chunks on prefixes: one extra query block
+    (2, 8, 8, 128, 1, 300, 128),             # decode rows only (MHA: G = 1 needs block 128)
+    (5, 16, 2, 64, 37, 37, 64),              # ragged, one partial block
+    (1, 64, 8, 128, 32768, 262144, 128),     # 32K chunk on a 256K context
+    (4, 8, 1, 128, 300, 300, 128),           # more query blocks would exceed the key blocks
+])
+def test_workspace_regions_follow_the_header(lib, S, Hq, Hkv, d, max_q, max_k, B):
+    """Every region of the workspace layout has at least the size the header
+    states for it, starts 256-byte aligned, and follows the previous one; the
+    padded block counts follow the header's formulas."""
+    P = base_params(num_seqs=S, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=d,
+                    total_q=S * max_q, total_k=S * max_k, max_seqlen_q=max_q,
+                    max_seqlen_k=max_k)
+    L = fp2.get_workspace_layout(P, B)
+    nkb = -(-max_k // B)
+    nqb = min((max_q + 2 * B - 2) // B, nkb)
+    nw = -(-nkb // 32)
+    assert (L.nqb_max, L.nkb_max, L.nw) == (nqb, nkb, nw)
+    regions = [(L.error_word, 16),
+               (L.kbar, 4 * S * Hkv * nkb * d), (L.vbar, 4 * S * Hkv * nkb * d),
+               (L.kbar_op, 2 * S * Hkv * nkb * d), (L.vbar_op, 2 * S * Hkv * nkb * d),
+               (L.scores, 4 * S * Hq * nqb * nkb), (L.kept_idx, 4 * S * Hq * nqb * nkb),
+               (L.kept_cnt, 4 * S * Hq * nqb), (L.kept_bits, 4 * S * Hq * nqb * nw)]
+    for (o, size), (o_next, _) in zip(regions, regions[1:] + [(L.total, 0)]):
+        assert o % 256 == 0
+        assert o_next - o >= size
+    assert fp2.workspace_size(P, B) == L.total
+
+
 @pytest.mark.parametrize("field,value,block,code", [
     ("num_kv_heads", 3, 128, fp2.FP2_ERR_INVALID_ARG),    # 32 % 3 != 0
     ("num_kv_heads", 2, 128, fp2.FP2_ERR_UNSUPPORTED),    # G = 16
