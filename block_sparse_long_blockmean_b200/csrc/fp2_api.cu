@@ -1,6 +1,10 @@
 // fp2_api.cu -- the C ABI of include/fp2.h: argument validation, workspace
 // layout, stream-ordered launches of the four kernels, the host-buffer
 // pipeline, status read-back and the host-side tau calibration utility.
+// fp2_prefill runs the method's four steps in the order the FlashPrefill V2
+// abstract gives them (block statistics, pattern discovery, dynamic
+// threshold, sparse attention with the mean correction); the host-buffer
+// pipeline and the tau utility are packaging with no counterpart there.
 #include <algorithm>
 #include <cmath>
 #include <cstring>

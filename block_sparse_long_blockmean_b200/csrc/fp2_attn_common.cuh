@@ -1,7 +1,10 @@
 // fp2_attn_common.cuh -- pieces shared by the two attention kernels:
 // tensor maps, the per-CTA work list (union of the G heads' kept blocks,
 // then the block-mean tiles that carry the correction), and the TMA issue of
-// one K/V (or mean) tile into a pipeline stage.
+// one K/V (or mean) tile into a pipeline stage.  The work list is the
+// PackGQA walk (FlashPrefill V2 popular explainer, section 2.2 kernel layer:
+// the G query heads of a KV head share each K/V tile); the mean tiles carry
+// the dropped blocks' constant term (same explainer, section 2.1).
 #pragma once
 
 #include <cuda_bf16.h>

@@ -1,4 +1,7 @@
-// fp2_seq.cuh -- per-sequence bookkeeping shared by the fp2 kernels.
+// fp2_seq.cuh -- per-sequence bookkeeping shared by the fp2 kernels: where a
+// call's query rows sit among the key blocks when the call is a chunk on a
+// resident prefix, of any length (FlashPrefill V2 popular explainer, section
+// 2.3 system layer: chunked prefill, chunks that mix prefill and decode rows).
 #pragma once
 
 #include "fp2_device.cuh"
