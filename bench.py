@@ -28,6 +28,7 @@ sys.path.insert(0, ROOT)
 METRIC = "128K prefill attn ms/layer & effective TFLOPS; % of B200 tensor peak"
 WORKLOAD_ID = 3
 DROP = 0.8
+DENSE_RUNS = 5
 
 
 def parse():
@@ -91,6 +92,31 @@ def recorded_traffic(dtype: str):
     if not m or not t or m.group(1) != attn_source_hash():
         return None
     return float(t.group(1))
+
+
+def fp8_gemm_peak_tflops(n: int = 8192, reps: int = 10):
+    """Live e4m3 GEMM throughput on this GPU (cuBLASLt through
+    torch._scaled_mm, n^3, bf16 output, best of `reps` back-to-back launches
+    after two warm-ups): the fp8 counterpart of the driver's measured bf16
+    GEMM peak.  None when the library call is unavailable."""
+    import torch
+    try:
+        a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        one = torch.ones((), device="cuda")
+        best = float("inf")
+        for it in range(reps + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            if it >= 2:
+                best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:
+        return None
 
 
 def measured_peaks():
@@ -298,15 +324,22 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
 
         dense = None
         if not args.no_dense:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            # the same attention kernel at tau = inf (every block kept): one
+            # warm-up launch, then the median of DENSE_RUNS timed launches
             fp2.mask(cu, math.inf, B, P)
             fp2.attn(q, k, v, pt, cu, None, B, dt, pr.out, P)  # warm
-            e0.record(stream)
-            fp2.attn(q, k, v, pt, cu, None, B, dt, pr.out, P)
-            e1.record(stream)
-            stream.synchronize()
-            dense = {"attn_ms": e0.elapsed_time(e1),
-                     "tflops": dense_flops(s.lens_q, s.lens_k, s.Hq, s.d) / (e0.elapsed_time(e1) * 1e-3) / 1e12}
+            d_ms = []
+            for _ in range(DENSE_RUNS):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fp2.attn(q, k, v, pt, cu, None, B, dt, pr.out, P)
+                e1.record(stream)
+                stream.synchronize()
+                d_ms.append(e0.elapsed_time(e1))
+            pr.check()
+            med = float(np.median(d_ms))
+            dense = {"attn_ms": med, "attn_ms_min": float(np.min(d_ms)), "runs": DENSE_RUNS,
+                     "tflops": dense_flops(s.lens_q, s.lens_k, s.Hq, s.d) / (med * 1e-3) / 1e12}
             fp2.mask(cu, tau, B, P)
 
         e2e = None
@@ -326,7 +359,7 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
             io = fp2.host_io(hq, hk, hv, hout, q, k, v, pr.out, cu_h, lk_h, upload_stream=up,
                              download_stream=down, num_chunks=args.e2e_chunks,
                              cu_seqlens_k_host=cuk_h)
-            nsteps = max(2, min(args.steps, 5))
+            nsteps = args.steps
             for it in range(nsteps + 1):
                 if it == 1:
                     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -600,25 +633,36 @@ def main():
     r = results[main_dt]
     total_ms, ms_per_layer = job_time(r["total_ms"], args.steps, world)
 
+    fp8_gemm = fp8_gemm_peak_tflops() if "fp8" in dtypes else None
+
     def summary(x):
         attn_ms = x["stage_ms"]["attn"]
         eff = x["kept_flops"] / (attn_ms * 1e-3) / 1e12
-        bf16_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        peak = bf16_peak * (2.0 if x["dtype"] == "fp8" else 1.0)
+        # burst peak: each step is tens of ms and the timed loop under a
+        # second, far from the seconds-long power-capped GEMM loop behind the
+        # sustained figure (kept beside it); fp8 = 2 x bf16 (nominal ratio)
+        ratio = 2.0 if x["dtype"] == "fp8" else 1.0
+        peak = peaks["bf16_tflops"] * ratio
+        peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * ratio
         out = {"attn_ms": attn_ms, "ms_per_layer": x["ms_per_step"],
                "eff_tflops_kept": eff,
                "eff_tflops_incl_correction": (x["kept_flops"] + x["corr_flops"]) / (attn_ms * 1e-3) / 1e12,
                "tensor_peak_frac_measured": eff / peak,
+               "tensor_peak_frac_measured_sustained": eff / peak_sus,
                "tensor_peak_frac_datasheet": eff / (2250.0 * (2.0 if x["dtype"] == "fp8" else 1.0)),
                "drop_fraction": x["drop_fraction"], "tau": x["tau"],
                "union_inflation": x["union_inflation"],
                "tensor_frac_executed_measured": eff * x["union_inflation"] / peak,
                "stage_ms": x["stage_ms"],
                "prefill_roofline_frac": (x["kept_flops"] / peak / 1e12) / (x["ms_per_step"] * 1e-3)}
+        if x["dtype"] == "fp8" and fp8_gemm:
+            out["fp8_gemm_tflops_measured"] = fp8_gemm
+            out["tensor_peak_frac_fp8_gemm"] = eff / fp8_gemm
         if x.get("mean_cache"):
             out["mean_cache"] = x["mean_cache"]
         if x["dense"]:
             out["dense_attn_ms"] = x["dense"]["attn_ms"]
+            out["dense_runs"] = x["dense"]["runs"]
             out["dense_tflops"] = x["dense"]["tflops"]
             out["speedup_vs_own_dense_attn"] = x["dense"]["attn_ms"] / attn_ms
         return out, peak
@@ -639,10 +683,12 @@ def main():
         "config": run_config(args, main_dt),
         "roofline": {"bound": "tensor", "achieved": eff, "peak": peak, "unit": "TFLOP/s",
                      "frac": eff / peak,
+                     "peak_sustained": s_main["eff_tflops_kept"] / s_main["tensor_peak_frac_measured_sustained"],
+                     "frac_sustained": s_main["tensor_peak_frac_measured_sustained"],
                      # the ncu figure is for the 128K layer's launch only
                      "traffic": recorded_traffic(main_dt) if args.workload == WORKLOAD_ID else None,
                      "kernel": "fp2_attn (attn_pair_kernel)",
-                     "peak_source": f"{peak_src} bf16_tflops_sustained" +
+                     "peak_source": f"{peak_src} bf16_tflops (burst; of measured)" +
                                     (" x2 (fp8/bf16 nominal ratio)" if main_dt == "fp8" else "")},
         "exp_roof": {"bound": "mufu", "achieved": exp_rate / 1e9, "peak": exp_peak / 1e9,
                      "unit": "Gexp/s", "frac": exp_rate / exp_peak,
