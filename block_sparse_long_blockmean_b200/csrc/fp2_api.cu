@@ -28,6 +28,8 @@ fp2_status check_params(const fp2_params* P, int block) {
         P->max_seqlen_q < 0 || P->max_seqlen_k < P->max_seqlen_q || P->max_seqlen_k < 1)
         return FP2_ERR_INVALID_ARG;
     if (P->num_q_heads % P->num_kv_heads != 0) return FP2_ERR_INVALID_ARG;
+    if (P->attn_kernel != 0 && P->attn_kernel != 1) return FP2_ERR_INVALID_ARG;
+    if (P->debug_withhold_k_item < 0) return FP2_ERR_INVALID_ARG;
     const int G = P->num_q_heads / P->num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return FP2_ERR_UNSUPPORTED;
     if (P->head_dim != 64 && P->head_dim != 128) return FP2_ERR_UNSUPPORTED;
@@ -133,6 +135,9 @@ fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_
     kp.group_masks = P->group_masks ? 1 : 0;
     kp.out_fp8 = P->out_dtype == FP2_FP8_E4M3;
     kp.out_scale = P->out_scale;
+    kp.attn_kernel = P->attn_kernel;
+    kp.wait_limit_ns = (unsigned long long)P->debug_wait_limit_us * 1000ull;
+    kp.withhold_k_item = P->debug_withhold_k_item;
     kp.cu_q = cu_seqlens;
     kp.cu_k = P->cu_seqlens_k ? P->cu_seqlens_k : cu_seqlens;
     kp.seqlens_k = P->seqlens_k;
@@ -285,12 +290,13 @@ fp2_status fp2_attn(const void* q, const void* k_cache, const void* v_cache,
     return cuda_status(e);
 }
 
-static fp2_status prefill_impl(const void* q, const void* k_cache, const void* v_cache,
-                               const int32_t* page_table, const int32_t* cu_seqlens, float tau,
-                               int block, fp2_dtype dtype, void* out, const fp2_params* params,
-                               const int32_t* block_table, int max_blocks_per_seq,
-                               float* mean_cache, int num_slots) {
-    KParams kp;
+// Every check fp2_prefill makes before it queues anything; fills kp.
+static fp2_status prefill_checks(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* page_table, const int32_t* cu_seqlens, float tau,
+                                 int block, fp2_dtype dtype, const void* out,
+                                 const fp2_params* params, const int32_t* block_table,
+                                 int max_blocks_per_seq, float* mean_cache, int num_slots,
+                                 KParams& kp) {
     fp2_status st = prepare(params, block, dtype, cu_seqlens, page_table, kp);
     if (st != FP2_OK) return st;
     if (mean_cache &&
@@ -301,8 +307,21 @@ static fp2_status prefill_impl(const void* q, const void* k_cache, const void* v
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return FP2_ERR_INVALID_ARG;
     if (std::isnan(tau)) return FP2_ERR_INVALID_ARG;
+    if (kp.total_q > 0 && !page_table && kp.total_k == 0) return FP2_ERR_INVALID_ARG;
+    return FP2_OK;
+}
+
+static fp2_status prefill_impl(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* page_table, const int32_t* cu_seqlens, float tau,
+                               int block, fp2_dtype dtype, void* out, const fp2_params* params,
+                               const int32_t* block_table, int max_blocks_per_seq,
+                               float* mean_cache, int num_slots) {
+    KParams kp;
+    fp2_status st = prefill_checks(q, k_cache, v_cache, page_table, cu_seqlens, tau, block, dtype,
+                                   out, params, block_table, max_blocks_per_seq, mean_cache,
+                                   num_slots, kp);
+    if (st != FP2_OK) return st;
     if (kp.total_q == 0) return FP2_OK;
-    if (!page_table && kp.total_k == 0) return FP2_ERR_INVALID_ARG;
     cudaStream_t s = stream_of(params);
     cudaError_t e = fp2::launch_blockmean(kp, k_cache, v_cache, s);
     kp.mean_cache = nullptr;  // only the block means use the cache
@@ -562,3 +581,14 @@ fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
 }
 
 }  // extern "C"
+
+namespace fp2 {
+fp2_status validate_prefill(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* page_table, const int32_t* cu_seqlens, float tau,
+                            int block, fp2_dtype dtype, const void* out,
+                            const fp2_params* params) {
+    KParams kp;
+    return prefill_checks(q, k_cache, v_cache, page_table, cu_seqlens, tau, block, dtype, out,
+                          params, nullptr, 0, nullptr, 0, kp);
+}
+}  // namespace fp2

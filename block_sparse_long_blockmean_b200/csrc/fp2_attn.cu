@@ -11,9 +11,10 @@
 //     logit q.kbar_j/sqrt(d) + ln(n_j) with n_j = B (dropped blocks are
 //     always full), value vbar_j.
 //
-// This one-tile kernel runs only when FP2_SINGLE_TILE is set (the two-tile
-// kernel of fp2_attn_pair.cu takes every problem otherwise); the tests keep
-// it as an independent second implementation of the same operator.
+// This one-tile kernel runs only when the caller asks for it
+// (fp2_params.attn_kernel = 1; the two-tile kernel of fp2_attn_pair.cu takes
+// every problem otherwise); the tests keep it as an independent second
+// implementation of the same operator.
 //
 // Work item = (sequence, KV head, query block i, slice tq): 128 tensor-core
 // rows = 128/G query tokens x the G query heads of the KV head (PackGQA: the
@@ -34,8 +35,6 @@
 //               (bf16 | e4m3) to shared memory in the 128-byte swizzle
 //               layout, and at the end normalises O and stores bf16 rows.
 // TMEM: S0 cols [0,128), S1 [128,256), O [256,256+d).
-#include <cstdlib>
-
 #include "fp2_attn_common.cuh"
 
 namespace fp2 {
@@ -96,6 +95,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
     const int hk = (rem / ntq) % p.Hkv;
     const int tq = rem % ntq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t wlim = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
 
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
@@ -155,7 +155,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             if (lane == 0) {
                 const int st = n & 1;
                 if (n >= 2 && !mbar_wait(&bars[B_KV_EMPTY + st], ((n - 2) >> 1) & 1, abort_flag,
-                                         kWaitLimitNs)) {
+                                         wlim)) {
                     set_error(p.err, kErrTimeout, kDetWaitBase + 0);
                     ok = false;
                 } else {
@@ -174,8 +174,8 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             // of the last two stages, whatever happened above
             volatile int no_abort = 0;
             for (int n = max(0, issued - 2); n < issued; ++n)
-                mbar_wait(&bars[B_KV_FULL + (n & 1)], (n >> 1) & 1, &no_abort, kWaitLimitNs);
-            mbar_wait(&bars[B_Q_FULL], 0, &no_abort, kWaitLimitNs);
+                mbar_wait(&bars[B_KV_FULL + (n & 1)], (n >> 1) & 1, &no_abort, wlim);
+            mbar_wait(&bars[B_Q_FULL], 0, &no_abort, wlim);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issue ---
@@ -184,16 +184,16 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             constexpr uint32_t idesc_qk = make_idesc(fmt, false, 128, BLK);
             constexpr uint32_t idesc_pv = make_idesc(fmt, true, 128, D);
             const uint32_t o_tmem = tmem + 256;
-            bool ok = mbar_wait(&bars[B_Q_FULL], 0, abort_flag, kWaitLimitNs);
+            bool ok = mbar_wait(&bars[B_Q_FULL], 0, abort_flag, wlim);
             if (!ok) set_error(p.err, kErrTimeout, kDetWaitBase + 1);
             tc_fence_after();
             for (int n = 0; ok && n <= n_items; ++n) {
                 if (n < n_items) {
                     const int st = n & 1;
-                    if (!mbar_wait(&bars[B_KV_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs) ||
+                    if (!mbar_wait(&bars[B_KV_FULL + st], (n >> 1) & 1, abort_flag, wlim) ||
                         (n >= 2 &&
                          !mbar_wait(&bars[B_S_FREE + st], ((n - 2) >> 1) & 1, abort_flag,
-                                    kWaitLimitNs))) {
+                                    wlim))) {
                         set_error(p.err, kErrTimeout, kDetWaitBase + 2);
                         ok = false;
                         break;
@@ -215,7 +215,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 if (n >= 1) {
                     const int m = n - 1;
                     const int stp = m & 1;
-                    if (!mbar_wait(&bars[B_P_READY], m & 1, abort_flag, kWaitLimitNs)) {
+                    if (!mbar_wait(&bars[B_P_READY], m & 1, abort_flag, wlim)) {
                         set_error(p.err, kErrTimeout, kDetWaitBase + 3);
                         ok = false;
                         break;
@@ -239,7 +239,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             // all MMAs of this thread complete before the CTA may release TMEM
             mma_commit(&bars[B_DRAIN]);
             volatile int no_abort = 0;
-            mbar_wait(&bars[B_DRAIN], 0, &no_abort, kWaitLimitNs);
+            mbar_wait(&bars[B_DRAIN], 0, &no_abort, wlim);
         }
     } else {
         // ------------------------------------------------ softmax warpgroup ---
@@ -284,7 +284,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 }
             }
             if (!__all_sync(0xffffffffu,
-                            mbar_wait(&bars[B_S_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs))) {
+                            mbar_wait(&bars[B_S_FULL + st], (n >> 1) & 1, abort_flag, wlim))) {
                 set_error(p.err, kErrTimeout, kDetWaitBase + 4);
                 ok = false;
                 break;
@@ -338,7 +338,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
             // PV of the previous item must be complete before P and O change
             if (n >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars[B_O_DONE], (n - 1) & 1,
-                                                             abort_flag, kWaitLimitNs))) {
+                                                             abort_flag, wlim))) {
                 set_error(p.err, kErrTimeout, kDetWaitBase + 5);
                 ok = false;
                 break;
@@ -400,7 +400,7 @@ attn_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
         }
         // ------------------------------------------------------- epilogue ---
         if (ok && __all_sync(0xffffffffu, mbar_wait(&bars[B_O_DONE], (n_items - 1) & 1,
-                                                    abort_flag, kWaitLimitNs))) {
+                                                    abort_flag, wlim))) {
             tc_fence_after();
             float inv = l > 0.f ? 1.f / l : 0.f;
             if (p.out_fp8) {
@@ -560,12 +560,11 @@ static cudaError_t launch_attn_t(const KParams& p, const void* q, const void* k,
 cudaError_t launch_attn_pair(const KParams& p, const void* q, const void* k, const void* v,
                              const uint32_t* kept_bits, void* out, cudaStream_t st);
 
-// Query blocks of at least 256 packed rows (G * block >= 256) go to the
-// two-tile kernel; smaller ones to the single-tile kernel above.
+// Every problem goes to the two-tile kernel unless the caller selected the
+// one-tile kernel above (KParams::attn_kernel = 1).
 cudaError_t launch_attn(const KParams& p, const void* q, const void* k, const void* v,
                         const uint32_t* kept_bits, void* out, cudaStream_t st) {
-    if (!getenv("FP2_SINGLE_TILE"))
-        return launch_attn_pair(p, q, k, v, kept_bits, out, st);
+    if (p.attn_kernel == 0) return launch_attn_pair(p, q, k, v, kept_bits, out, st);
     if (p.fp8) {
         if (p.d == 128 && p.B == 128) return launch_attn_t<128, 128, true>(p, q, k, v, kept_bits, out, st);
         return cudaErrorInvalidValue;

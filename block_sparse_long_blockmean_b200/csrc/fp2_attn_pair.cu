@@ -56,7 +56,7 @@ struct PairCfg {
     static constexpr int OFF_BAR = OFF_V + S * KV_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + 256;
     static constexpr int OFF_RING = OFF_MISC + 64;  // page ids of upcoming items
-    static constexpr int OFF_ITEMS = OFF_RING + kPageRing * kMaxBoxes * 4;
+    static constexpr int OFF_ITEMS = OFF_RING + 2 * kPageRing * kMaxBoxes * 4;  // K and V rings
     static_assert(P_COLS % 32 == 0, "P row must be whole 32-column TMEM stores");
     // pairs (of every 4) whose exp2 runs on the FMA pipe: the fp8 MMA is twice
     // as fast, so more of the exp2 work moves off the MUFU unit there
@@ -67,7 +67,22 @@ struct PairCfg {
 #define FP2_EMU_PAIRS_BF16 0
 #endif
     static constexpr int kEmuPairs = FP8 ? FP2_EMU_PAIRS_FP8 : FP2_EMU_PAIRS_BF16;
+    // polynomial degree of the FMA-pipe exp2: e4m3 probabilities need less
+#ifndef FP2_EMU_DEG_FP8
+#define FP2_EMU_DEG_FP8 2
+#endif
+    static constexpr int kEmuDeg = FP8 ? FP2_EMU_DEG_FP8 : 3;
 };
+
+// FMA-pipe exp2 with the clamp folded into a saturating FMA (exp2_sat_poly2)
+// instead of two fmax on the integer/ALU pipe
+#ifndef FP2_EXP_SAT
+#define FP2_EXP_SAT 0
+#endif
+
+#ifndef FP2_SPLIT_PRODUCER
+#define FP2_SPLIT_PRODUCER 1
+#endif
 
 // K and V have separate rings: K(n) is free once QK_B(n) has run, V(n) only
 // after PV_B(n) -- a full MMA pair later -- so each stream refills as soon as
@@ -110,6 +125,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
     const int hk = xq ? rem % p.Hkv : (rem / npair) % p.Hkv;
     const int pr = xq ? 0 : rem % npair;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t wlim = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
 
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
@@ -128,7 +144,8 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     if (threadIdx.x == 0) {
         for (int k = 0; k < PB_COUNT; ++k)
-            mbar_init(&bars[k], (k == PB_P_READY || k == PB_P_READY + 1) ? 128u : 1u);
+            mbar_init(&bars[k], (k == PB_P_READY || k == PB_P_READY + 1) ? 128u
+                                : (FP2_SPLIT_PRODUCER && k < PB_K_EMPTY) ? 2u : 1u);
         misc[1] = 0;
         fence_mbar_init();
         // both Q tiles right away: their latency overlaps the kept-bit loads
@@ -159,6 +176,79 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     if (warp >= 8) {
       regs_decrease<56>();
+#if FP2_SPLIT_PRODUCER
+      if (warp == 8 || warp == 10) {
+        // --------------------------------------------------------- producers ---
+        // warp 8 issues the K ring, warp 10 the V ring; each warp resolves
+        // the page ids of its own items 32 at a time into its own page ring,
+        // and its lane 0 waits and issues.  Step n of the pipeline is K(n)
+        // and V(n-1); KV_FULL[n % 2] counts one arrival from each warp per
+        // step, each arriving together with the bytes it will land (a warp
+        // with no tile at step n -- K at n = n_items, V at n = 0 -- arrives
+        // alone), so a phase cannot complete before both warps registered
+        // their bytes.  Before arriving at step n >= 2 a warp makes sure
+        // step n-2 (same barrier, previous phase) has completed: implied by
+        // its EMPTY wait (K(n) waits for QK_B(n-2), V(n-1) for PV_B(n-3),
+        // both issued after the MMA thread saw step n-2 complete), and
+        // waited for explicitly where no EMPTY wait implies it.
+        const bool is_k = warp == 8;
+        int* pring = reinterpret_cast<int*>(smem + C::OFF_RING) +
+                     (is_k ? 0 : kPageRing * kMaxBoxes);
+        const CUtensorMap* map = is_k ? &maps.k : &maps.v;
+        const CUtensorMap* mean_map = is_k ? &maps.kb : &maps.vb;
+        const uint32_t ring_s = sbase + (is_k ? C::OFF_K : C::OFF_V);
+        uint64_t* empty = &bars[is_k ? PB_K_EMPTY : PB_V_EMPTY];
+        if (lane == 0) prefetch_tmap(map);
+        int last = -1;  // last step at which this warp arrived on KV_FULL
+        bool ok = true;
+        for (int n = 0; n <= n_items; ++n) {
+            const int m = is_k ? n : n - 1;  // the item this warp loads at step n
+            const bool has = m >= 0 && m < n_items;
+            if (has && m % 32 == 0) fill_page_ring<BLK>(p, s, b, items, n_items, m, pring);
+            if (lane == 0) {
+                uint64_t* full = &bars[PB_KV_FULL + n % C::S];
+                const int st = m & 1;
+                const bool implied = has && m >= C::S;  // the EMPTY wait implies step n-2
+                if (n >= 2 && !implied &&
+                    !mbar_wait(full, ((n - 2) / C::S) & 1, abort_flag, wlim)) {
+                    set_error(p.err, kErrTimeout, kDetWaitBase + 8);
+                    ok = false;
+                } else if (!has) {
+                    mbar_arrive(full);
+                    last = n;
+                } else if (is_k && p.withhold_k_item == m + 1) {
+                    ok = false;  // test knob: K(m) is never loaded nor announced
+                } else if (m >= C::S && !mbar_wait(&empty[st], ((m - C::S) / C::S) & 1,
+                                                   abort_flag, wlim)) {
+                    set_error(p.err, kErrTimeout, kDetWaitBase + 0);
+                    ok = false;
+                } else {
+                    issue_tile_load<D, BLK, FP8>(p, map, mean_map, s, b, hk, items[m],
+                                                 pring + (m % kPageRing) * kMaxBoxes,
+                                                 ring_s + st * C::KV_BYTES, full, true);
+                    last = n;
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        }
+        if (lane == 0) {
+            // never leave with copies in flight: wait for the phases of the
+            // last two steps this warp arrived at.  Its copies of earlier
+            // steps landed before it could arrive at these (the step n-2 rule
+            // above), and no later phase of either barrier can complete
+            // without this warp, so a parity wait cannot see a stale phase.
+            // In a normal run both warps arrive at every step and these waits
+            // end at once; one that runs out is recorded (after an abort the
+            // first error is already there and a partner that stopped early
+            // only costs the limit).
+            volatile int no_abort = 0;
+            bool drained = true;
+            for (int n = max(0, last - 1); n <= last; ++n)
+                drained &= mbar_wait(&bars[PB_KV_FULL + n % C::S], (n / C::S) & 1, &no_abort, wlim);
+            if (is_k) drained &= mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, wlim);
+            if (!drained) set_error(p.err, kErrTimeout, kDetWaitBase + 12);
+        }
+#else
       if (warp == 8) {
         // ---------------------------------------------------------- producer ---
         // the whole warp resolves page ids 32 items at a time; lane 0 waits
@@ -180,7 +270,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 if (n < n_items) {
                     const int st = n % C::S;
                     if (n >= C::S && !mbar_wait(&bars[PB_K_EMPTY + st], ((n - C::S) / C::S) & 1,
-                                                abort_flag, kWaitLimitNs)) {
+                                                abort_flag, wlim)) {
                         set_error(p.err, kErrTimeout, kDetWaitBase + 0);
                         ok = false;
                     } else {
@@ -195,7 +285,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 if (ok && n >= 1) {
                     const int m = n - 1, st = m % C::S;
                     if (m >= C::S && !mbar_wait(&bars[PB_V_EMPTY + st], ((m - C::S) / C::S) & 1,
-                                                abort_flag, kWaitLimitNs)) {
+                                                abort_flag, wlim)) {
                         set_error(p.err, kErrTimeout, kDetWaitBase + 0);
                         ok = false;
                         // K(n) went without an arrival: arrive so that the
@@ -216,21 +306,22 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             // never leave with copies in flight: the last steps that issued any
             volatile int no_abort = 0;
             for (int n = max(0, steps - C::S); n < steps; ++n)
-                mbar_wait(&bars[PB_KV_FULL + n % C::S], (n / C::S) & 1, &no_abort, kWaitLimitNs);
-            mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, kWaitLimitNs);
+                mbar_wait(&bars[PB_KV_FULL + n % C::S], (n / C::S) & 1, &no_abort, wlim);
+            mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, wlim);
         }
+#endif
       } else if (warp == 9 && lane == 0) {
         // -------------------------------------------------------------- MMA ---
             constexpr uint32_t fmt = FP8 ? 0u : 1u;
             constexpr uint32_t idesc_qk = make_idesc(fmt, false, 128, BLK);
             constexpr uint32_t idesc_pv = make_idesc(fmt, true, 128, D);
-            bool ok = mbar_wait(&bars[PB_Q_FULL], 0, abort_flag, kWaitLimitNs);
+            bool ok = mbar_wait(&bars[PB_Q_FULL], 0, abort_flag, wlim);
             if (!ok) set_error(p.err, kErrTimeout, kDetWaitBase + 1);
             tc_fence_after();
             for (int n = 0; ok && n <= n_items; ++n) {
                 const int st = n & 1;
                 // K(n) and V(n-1)
-                if (!mbar_wait(&bars[PB_KV_FULL + st], (n >> 1) & 1, abort_flag, kWaitLimitNs)) {
+                if (!mbar_wait(&bars[PB_KV_FULL + st], (n >> 1) & 1, abort_flag, wlim)) {
                     set_error(p.err, kErrTimeout, kDetWaitBase + 2);
                     ok = false;
                     break;
@@ -239,7 +330,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 for (int x = 0; x < 2; ++x) {
                     if (n >= 1) {
                         const int m = n - 1;
-                        if (!mbar_wait(&bars[PB_P_READY + x], m & 1, abort_flag, kWaitLimitNs)) {
+                        if (!mbar_wait(&bars[PB_P_READY + x], m & 1, abort_flag, wlim)) {
                             set_error(p.err, kErrTimeout, kDetWaitBase + 3);
                             ok = false;
                             break;
@@ -280,7 +371,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             }
             mma_commit(&bars[PB_DRAIN]);
             volatile int no_abort = 0;
-            mbar_wait(&bars[PB_DRAIN], 0, &no_abort, kWaitLimitNs);
+            mbar_wait(&bars[PB_DRAIN], 0, &no_abort, wlim);
       }
     } else {
         regs_increase<224>();
@@ -334,7 +425,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 }
             }
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[PB_S_FULL + X], n & 1, abort_flag,
-                                                   kWaitLimitNs))) {
+                                                   wlim))) {
                 set_error(p.err, kErrTimeout, kDetWaitBase + 4);
                 ok = false;
                 break;
@@ -400,6 +491,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 // a row that takes no part gets offset -inf: every p is 0
                 const float c0 = live ? bias - m_used : -INFINITY;
                 const float2 k2 = make_float2(sl2, sl2), c2 = make_float2(c0, c0);
+                const float k128 = sl2 * (1.f / 128.f), c128 = (c0 + 120.f) * (1.f / 128.f);
                 float2 a0 = make_float2(0.f, 0.f), a1 = a0;
                 // of every 4 pairs, the last kEmuPairs go to the FMA pipe
                 // (exp2_poly2), the rest to MUFU ex2: the two units share the load
@@ -407,9 +499,16 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 for (int c = 0; c < BLK / 2; c += 4) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const float2 e = ffma2(xv[c + u], k2, c2);
-                        xv[c + u] = (u >= 4 - C::kEmuPairs) ? exp2_poly2(e)
-                                                             : make_float2(ex2(e.x), ex2(e.y));
+                        if (u >= 4 - C::kEmuPairs) {
+#if FP2_EXP_SAT
+                            xv[c + u] = exp2_sat_poly2<C::kEmuDeg>(xv[c + u], k128, c128);
+#else
+                            xv[c + u] = exp2_poly2<C::kEmuDeg>(ffma2(xv[c + u], k2, c2));
+#endif
+                        } else {
+                            const float2 e = ffma2(xv[c + u], k2, c2);
+                            xv[c + u] = make_float2(ex2(e.x), ex2(e.y));
+                        }
                         if (u & 1) a1 = fadd2(a1, xv[c + u]);
                         else a0 = fadd2(a0, xv[c + u]);
                     }
@@ -436,7 +535,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 // V(n) loads one step behind K(n): let it land before zeroing
                 // (V(n+2) cannot reuse the slot before this warpgroup's P(n))
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[PB_KV_FULL + ((n + 1) & 1)], ((n + 1) >> 1) & 1,
-                                                       abort_flag, kWaitLimitNs))) {
+                                                       abort_flag, wlim))) {
                     set_error(p.err, kErrTimeout, kDetWaitBase + 7);
                     ok = false;
                     break;
@@ -450,7 +549,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             mbar_arrive(&bars[PB_P_READY + X]);
         }
         if (ok && __all_sync(0xffffffffu, mbar_wait(&bars[PB_O_FINAL + X], 0, abort_flag,
-                                                    kWaitLimitNs))) {
+                                                    wlim))) {
             tc_fence_after();
             float inv = l > 0.f ? 1.f / l : 0.f;
             if (p.out_fp8) {

@@ -48,6 +48,14 @@ struct KParams {
     float* mean_cache;
     const int32_t* block_table;
     int max_blocks, num_slots;
+    // limit of every pipeline wait of the attention kernels, in ns (0: the
+    // default 2 s); test-only knob of the bounded-wait error path
+    unsigned long long wait_limit_ns;
+    // > 0: the attention producer withholds the K tile of that work item
+    // (1-based) in every CTA, so the consumer's bounded wait runs out
+    // (test-only; 0 in every normal call)
+    int withhold_k_item;
+    int attn_kernel;           // 0: two-tile kernel, 1: one-tile kernel
 };
 
 // Detail codes stored beside an error code.

@@ -59,6 +59,9 @@ class Params(ctypes.Structure):
         ("group_masks", ctypes.c_int),
         ("out_dtype", ctypes.c_int),
         ("out_scale", ctypes.c_void_p),
+        ("attn_kernel", ctypes.c_int),
+        ("debug_wait_limit_us", ctypes.c_uint),
+        ("debug_withhold_k_item", ctypes.c_int),
     ]
 
 
@@ -128,6 +131,7 @@ SIGNATURES = {
                                 _PP]),
     "fp2_workspace_init": (ctypes.c_int, [_PP]),
     "fp2_get_status": (ctypes.c_int, [_PP, ctypes.POINTER(ctypes.c_uint32)]),
+    "fp2_noalloc_get_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "fp2_calibrate_tau": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_float, _PP,
                                          ctypes.POINTER(ctypes.c_float)]),
     "fp2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -278,6 +282,17 @@ def get_status(params: Params) -> tuple[int, int]:
     return int(st), int(det.value)
 
 
+def noalloc_get_status(stream=None) -> tuple[int, int]:
+    """Device-side status of the last fp2_prefill_noalloc call(s) on the
+    current device; synchronises ``stream`` (default: torch's current one)."""
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream().cuda_stream
+    det = ctypes.c_uint32(0)
+    st = lib().fp2_noalloc_get_status(stream, ctypes.byref(det))
+    return int(st), int(det.value)
+
+
 def calibrate_tau(cu_seqlens, block: int, target_drop: float, params: Params) -> float:
     t = ctypes.c_float(0.0)
     _check(lib().fp2_calibrate_tau(_ptr(cu_seqlens), block, float(target_drop),
@@ -334,7 +349,7 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
                  page_table=None, page_size: int = 0, q_scale=None, k_scale=None,
                  v_scale=None, out=None, stream=None, workspace=None,
                  group_masks: bool = False, out_dtype: int = FP2_BF16,
-                 out_scale=None) -> Problem:
+                 out_scale=None, attn_kernel: int = 0) -> Problem:
     """Builds fp2_params for device tensors and allocates the workspace and
     the bf16 output with torch (allocation only)."""
     import torch
@@ -357,6 +372,7 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
     P.group_masks = 1 if group_masks else 0
     P.out_dtype = out_dtype
     P.out_scale = _ptr(out_scale)
+    P.attn_kernel = int(attn_kernel)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
     P.stream = stream

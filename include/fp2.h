@@ -50,8 +50,8 @@
  *
  * Kernel choice: the two-tile attention kernel runs every problem (two
  * 128-row tiles of one query block when G * block >= 256, else two adjacent
- * query blocks); the environment variable FP2_SINGLE_TILE=1 forces the
- * one-tile kernel instead (tests).
+ * query blocks); params->attn_kernel = 1 selects the one-tile kernel instead
+ * (a second, independent implementation of the same step, kept for tests).
  *
  * Errors: argument errors are returned synchronously before any launch.
  * CUDA launch errors return FP2_ERR_CUDA.  Problems only the device can see
@@ -111,6 +111,17 @@ typedef struct fp2_params {
     const float* out_scale;    /* device [Hq], e4m3 output only.  NULL with FP8 inputs: the
                                   KV head's v_scale (|O| <= max|V|, so it never saturates);
                                   required with BF16 inputs */
+    int attn_kernel;           /* 0 (default): the two-tile attention kernel.  1: the one-tile
+                                  kernel (same results within rounding; for tests) */
+    unsigned int debug_wait_limit_us; /* 0 (default): every pipeline wait inside the
+                                  attention kernel gives up after 2 s, records
+                                  FP2_ERR_TIMEOUT and ends its CTA cleanly.  > 0: after this
+                                  many microseconds instead (tests of that path) */
+    int debug_withhold_k_item; /* 0 (default).  > 0, tests only: the two-tile kernel's
+                                  producer never loads the K tile of that work item
+                                  (1-based) in any CTA, so the consumer's bounded wait runs
+                                  out and the call records FP2_ERR_TIMEOUT; the output is
+                                  then undefined.  Never set in normal use */
 } fp2_params;
 
 /* Offsets (bytes from params->workspace) of the intermediates, for callers
@@ -294,12 +305,24 @@ fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
  *  - Every call shares the one array and leaves its contents behind; calls
  *    whose work overlaps on the GPU (other streams, other host threads) race
  *    on it, so the caller must serialise them.
- *  - The array's error word is cleared at the start of each call; device-side
- *    errors of this call cannot be read with fp2_get_status. */
+ *  - Arguments are checked exactly as fp2_prefill checks them, before the
+ *    array is touched: a rejected call queues nothing.
+ *  - The array's error word is cleared at the start of each call; the
+ *    device-side errors of the last call are read with
+ *    fp2_noalloc_get_status (not fp2_get_status, which reads a caller's
+ *    workspace). */
 fp2_status fp2_prefill_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* page_table, const int32_t* cu_seqlens,
                                float tau, int block, fp2_dtype dtype, void* out,
                                const fp2_params* params);
+
+/* fp2_get_status for fp2_prefill_noalloc: synchronises `stream` (a
+ * cudaStream_t; NULL = the legacy default stream) and returns the first
+ * device-side error recorded in the library-owned array of the current device
+ * since it was last cleared (FP2_OK if none), then clears it.  *detail (host,
+ * may be NULL) receives the error's detail word.  The paper has no
+ * counterpart; packaging, like fp2_prefill_noalloc itself. */
+fp2_status fp2_noalloc_get_status(void* stream, uint32_t* detail);
 
 /* Static string naming a status code. */
 const char* fp2_status_string(fp2_status status);

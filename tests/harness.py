@@ -16,7 +16,8 @@ NEAR_THRESHOLD = 1e-3
 
 
 def problem(inp: synth.Inputs, dev: str = "cuda", out_fill: float | None = None,
-            ws_fill: int | None = None, group_masks: bool = False) -> fp2.Problem:
+            ws_fill: int | None = None, group_masks: bool = False,
+            attn_kernel: int = 0) -> fp2.Problem:
     s = inp.shape
     dtype = fp2.FP2_FP8_E4M3 if s.dtype == "fp8" else fp2.FP2_BF16
     q = inp.q.to(dev)
@@ -35,7 +36,7 @@ def problem(inp: synth.Inputs, dev: str = "cuda", out_fill: float | None = None,
                           seqlens_k=lk, cu_seqlens_k=cu_k, page_table=pt,
                           page_size=s.page_size or (k.shape[1] if inp.paged else 0),
                           q_scale=sc[0], k_scale=sc[1], v_scale=sc[2], out=out,
-                          group_masks=group_masks)
+                          group_masks=group_masks, attn_kernel=attn_kernel)
     if ws_fill is not None:
         pr.workspace.fill_(ws_fill)
         fp2.workspace_init(pr.params)

@@ -249,14 +249,14 @@ def test_calibrate_tau_matches_target():
 
 @pytest.mark.parametrize("name", ["tiny_1k_d64_b64", "varlen_paged64_fp8", "chunk_prefix_g8",
                                   "ragged_2k_g4"])
-def test_single_tile_kernel_on_large_groups(name, monkeypatch):
-    """FP2_SINGLE_TILE=1 routes G*block >= 256 problems to the one-tile kernel
-    too, so both attention kernels are checked on the same cases."""
-    monkeypatch.setenv("FP2_SINGLE_TILE", "1")
+def test_single_tile_kernel_on_large_groups(name):
+    """fp2_params.attn_kernel = 1 routes G*block >= 256 problems to the
+    one-tile kernel too, so both attention kernels are checked on the same
+    cases."""
     inp = make_inputs(name)
     orc = H.oracle_scores(inp)
     tau = H.pick_tau(orc, inp.shape.drop)
-    pr = H.problem(inp, out_fill=float("nan"))
+    pr = H.problem(inp, out_fill=float("nan"), attn_kernel=1)
     pr.prefill(tau)
     pr.check()
     for b in range(inp.num_seqs):

@@ -56,16 +56,12 @@ def random_case(k: int):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("k", range(N_CASES))
-def test_random_problem(k, monkeypatch):
+def test_random_problem(k):
     kw, force_single = random_case(k)
-    if force_single:
-        monkeypatch.setenv("FP2_SINGLE_TILE", "1")
-    else:
-        monkeypatch.delenv("FP2_SINGLE_TILE", raising=False)
     inp = synth.make_inputs(H.small_shape(**kw))
     orc = H.oracle_scores(inp)
     tau = H.pick_tau(orc, kw["drop"])
-    pr = H.problem(inp, out_fill=float("nan"), ws_fill=0xFF)
+    pr = H.problem(inp, out_fill=float("nan"), ws_fill=0xFF, attn_kernel=int(force_single))
     pr.prefill(tau)
     pr.check()
     got = H.gpu_bits(pr, inp)
