@@ -47,6 +47,9 @@ def parse():
                          "229376-token paged prefix (also times the block-mean cache)")
     ap.add_argument("--out-fp8", action="store_true",
                     help="e4m3 output (fp8 runs; default scale: the KV head's v_scale)")
+    ap.add_argument("--kv-scales", default="head", choices=["head", "block"],
+                    help="e4m3 K/V scales: one per head, or one per (sequence, key block, "
+                         "head) given as factors of the per-head scale (fp8 runs only)")
     ap.add_argument("--group-masks", action="store_true",
                     help="one mask per KV group (variant) instead of one per query head")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -244,6 +247,8 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
 
     dev = torch.device("cuda", torch.cuda.current_device())
     shape = synth.workload(args.workload, dtype_name)
+    if dtype_name == "fp8":
+        shape.kv_scales = args.kv_scales
     t0 = time.time()
     inp = synth.make_inputs(shape)
     gen_s = time.time() - t0
@@ -257,13 +262,16 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
     pt = inp.page_table.to(dev) if inp.paged else None
     cuk = None if inp.paged else inp.cu_seqlens_k.to(dev)
     sc = [x.to(dev) if x is not None else None for x in (inp.q_scale, inp.k_scale, inp.v_scale)]
+    fac = [x.contiguous().to(dev) if x is not None else None
+           for x in (inp.k_block_factor, inp.v_block_factor)]
     stream = torch.cuda.Stream(dev)
     pr = fp2.make_problem(q, k, v, cu, Hq=s.Hq, Hkv=s.Hkv, d=s.d, block=s.B, dtype=dt,
                           max_seqlen_q=max(s.lens_q), max_seqlen_k=max(s.lens_k),
                           seqlens_k=lk, cu_seqlens_k=cuk, page_table=pt,
                           page_size=k.shape[1] if inp.paged else 0, q_scale=sc[0],
                           k_scale=sc[1], v_scale=sc[2], stream=stream.cuda_stream,
-                          group_masks=args.group_masks,
+                          group_masks=args.group_masks, k_block_factor=fac[0],
+                          v_block_factor=fac[1],
                           out_dtype=fp2.FP2_FP8_E4M3 if (args.out_fp8 and dtype_name == "fp8")
                           else fp2.FP2_BF16)
     P = pr.params
@@ -399,7 +407,8 @@ def run_gpu(args, rank, world, dtype_name, stream_timing=True, want_cpu=False):
                                     max_seqlen_q=max(s.lens_k), max_seqlen_k=max(s.lens_k),
                                     seqlens_k=lk, page_table=pt, page_size=k.shape[1],
                                     q_scale=sc[0], k_scale=sc[1], v_scale=sc[2],
-                                    stream=stream.cuda_stream)
+                                    stream=stream.cuda_stream, k_block_factor=fac[0],
+                                    v_block_factor=fac[1])
             fill.params.total_q = int(sum(s.lens_k))
             fp2.blockmean_cached(k, v, pt, cu_full, table, max(nblk), cache, slots, B, dt,
                                  fill.params)
@@ -533,6 +542,8 @@ def run_config(args, dtype_name: str) -> dict:
             "l2": f"inputs ({in_bytes / 1e9:.2f} GB) larger than L2; no flush",
             "per_gpu": "one independent layer per GPU",
             "masks": "per KV group (variant)" if args.group_masks else "per query head",
+            "kv_scales": ("per key block (fp8 run)" if getattr(args, "kv_scales", "head") == "block"
+                          else "per head"),
             "output": "e4m3 for the fp8 run" if args.out_fp8 else "bf16"}
 
 

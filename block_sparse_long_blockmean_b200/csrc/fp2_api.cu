@@ -54,10 +54,12 @@ fp2_status check_dtype(const fp2_params* P, int block, fp2_dtype dtype) {
     if (P->out_dtype != FP2_BF16 && P->out_dtype != FP2_FP8_E4M3) return FP2_ERR_INVALID_ARG;
     if (P->out_dtype == FP2_FP8_E4M3 && dtype == FP2_BF16 && !P->out_scale)
         return FP2_ERR_INVALID_ARG;
-    if (dtype == FP2_BF16) return FP2_OK;
+    if (dtype == FP2_BF16) return (P->k_block_factor || P->v_block_factor) ? FP2_ERR_INVALID_ARG : FP2_OK;
     if (dtype != FP2_FP8_E4M3) return FP2_ERR_INVALID_ARG;
     if (P->head_dim != 128 || block != 128) return FP2_ERR_UNSUPPORTED;
     if (!P->q_scale || !P->k_scale || !P->v_scale) return FP2_ERR_INVALID_ARG;
+    if (!P->k_block_factor != !P->v_block_factor) return FP2_ERR_INVALID_ARG;
+    if (P->k_block_factor && P->attn_kernel != 0) return FP2_ERR_UNSUPPORTED;
     return FP2_OK;
 }
 
@@ -95,11 +97,14 @@ void layout_of(const fp2_params* P, int block, fp2_workspace_layout* L) {
 }
 
 // Validates what every entry point needs and fills the kernel parameters.
+// Entry points that take no dtype (mask, tau calibration) pass has_dtype =
+// false: the input and output formats are then not theirs to check.
 fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_t* cu_seqlens,
-                   const int32_t* page_table, KParams& kp, bool uses_kv = true) {
+                   const int32_t* page_table, KParams& kp, bool uses_kv = true,
+                   bool has_dtype = true) {
     fp2_status st = check_params(P, block);
     if (st != FP2_OK) return st;
-    if ((st = check_dtype(P, block, dtype)) != FP2_OK) return st;
+    if (has_dtype && (st = check_dtype(P, block, dtype)) != FP2_OK) return st;
     if ((st = check_kv(P, block, page_table)) != FP2_OK) return st;
     if (!cu_seqlens) return FP2_ERR_INVALID_ARG;
     fp2_workspace_layout L;
@@ -138,6 +143,8 @@ fp2_status prepare(const fp2_params* P, int block, fp2_dtype dtype, const int32_
     kp.attn_kernel = P->attn_kernel;
     kp.wait_limit_ns = (unsigned long long)P->debug_wait_limit_us * 1000ull;
     kp.withhold_k_item = P->debug_withhold_k_item;
+    kp.kb_fac = P->k_block_factor;
+    kp.vb_fac = P->v_block_factor;
     kp.cu_q = cu_seqlens;
     kp.cu_k = P->cu_seqlens_k ? P->cu_seqlens_k : cu_seqlens;
     kp.seqlens_k = P->seqlens_k;
@@ -266,7 +273,7 @@ fp2_status fp2_score(const void* q, const int32_t* cu_seqlens, int block, fp2_dt
 
 fp2_status fp2_mask(const int32_t* cu_seqlens, float tau, int block, const fp2_params* params) {
     KParams kp;
-    fp2_status st = prepare(params, block, FP2_BF16, cu_seqlens, nullptr, kp, false);
+    fp2_status st = prepare(params, block, FP2_BF16, cu_seqlens, nullptr, kp, false, false);
     if (st != FP2_OK) return st;
     if (std::isnan(tau)) return FP2_ERR_INVALID_ARG;
     return cuda_status(fp2::launch_mask(kp, tau, stream_of(params)));
@@ -373,7 +380,7 @@ fp2_status fp2_get_status(const fp2_params* params, uint32_t* detail) {
 fp2_status fp2_calibrate_tau(const int32_t* cu_seqlens, int block, float target_drop,
                              const fp2_params* params, float* tau_out) {
     KParams kp;
-    fp2_status st = prepare(params, block, FP2_BF16, cu_seqlens, nullptr, kp, false);
+    fp2_status st = prepare(params, block, FP2_BF16, cu_seqlens, nullptr, kp, false, false);
     if (st != FP2_OK) return st;
     if (!tau_out || !(target_drop >= 0.f && target_drop <= 1.f)) return FP2_ERR_INVALID_ARG;
     cudaStream_t s = stream_of(params);

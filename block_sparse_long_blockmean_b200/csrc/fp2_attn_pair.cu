@@ -64,7 +64,7 @@ struct PairCfg {
 #define FP2_EMU_PAIRS_FP8 1
 #endif
 #ifndef FP2_EMU_PAIRS_BF16
-#define FP2_EMU_PAIRS_BF16 0
+#define FP2_EMU_PAIRS_BF16 1
 #endif
     static constexpr int kEmuPairs = FP8 ? FP2_EMU_PAIRS_FP8 : FP2_EMU_PAIRS_BF16;
     // polynomial degree of the FMA-pipe exp2: e4m3 probabilities need less
@@ -75,10 +75,13 @@ struct PairCfg {
 };
 
 // FMA-pipe exp2 with the clamp folded into a saturating FMA (exp2_sat_poly2)
-// instead of two fmax on the integer/ALU pipe
+// instead of two fmax on the ALU pipe.  Its range ends at exponent 8, which
+// the lazy rescale guarantees: every exponent is x * sl2 + bias - m_used with
+// the row's maximum at most kRescaleLog2 above m_used.
 #ifndef FP2_EXP_SAT
-#define FP2_EXP_SAT 0
+#define FP2_EXP_SAT 1
 #endif
+static_assert(!FP2_EXP_SAT || kRescaleLog2 <= 8.f, "exp2_sat_poly2 covers exponents up to 8");
 
 #ifndef FP2_SPLIT_PRODUCER
 #define FP2_SPLIT_PRODUCER 1
@@ -404,6 +407,20 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             const int item = items[n];
             bool live;                  // this row takes part in this item
             float bias = 0.f;
+            // a cache quantised per key block: the block's K factor scales its
+            // logits (sl2i), its V factor is folded into P before the e4m3
+            // rounding as log2 fv in the exponent (lvi <= 0), and the row sum
+            // takes the unscaled p (inv_fv).  Mean tiles are in per-head units.
+            float sl2i = sl2, lvi = 0.f, inv_fv = 1.f;
+            if constexpr (FP8) {
+                if (p.kb_fac && item >= 0) {
+                    const size_t fi = ((size_t)b * p.nkb_max + item) * p.Hkv + hk;
+                    const float fk = __ldg(p.kb_fac + fi), fv = __ldg(p.vb_fac + fi);
+                    sl2i = sl2 * fk;
+                    lvi = __log2f(fv);
+                    inv_fv = 1.f / fv;
+                }
+            }
             uint32_t dropped[BLK / 32];  // mean tiles: the row's dropped blocks
             if (item >= 0) {
                 live = row_ok && ((hb[item >> 5] >> (item & 31)) & 1u);
@@ -462,7 +479,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                     else m3 = fmaxf(m3, x[c + 6]);
                 }
                 mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-                if (mx != -INFINITY) mx = fmaf(mx, sl2, bias);
+                if (mx != -INFINITY) mx = fmaf(mx, sl2i, bias);
             }
             float alpha = 1.f;
             bool rescale = false;
@@ -489,12 +506,13 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             float sum = 0.f;
             {
                 // a row that takes no part gets offset -inf: every p is 0
-                const float c0 = live ? bias - m_used : -INFINITY;
-                const float2 k2 = make_float2(sl2, sl2), c2 = make_float2(c0, c0);
-                const float k128 = sl2 * (1.f / 128.f), c128 = (c0 + 120.f) * (1.f / 128.f);
+                const float c0 = live ? bias - m_used + lvi : -INFINITY;
+                const float2 k2 = make_float2(sl2i, sl2i), c2 = make_float2(c0, c0);
+                const float k128 = sl2i * (1.f / 128.f), c128 = (c0 + 120.f) * (1.f / 128.f);
                 float2 a0 = make_float2(0.f, 0.f), a1 = a0;
                 // of every 4 pairs, the last kEmuPairs go to the FMA pipe
-                // (exp2_poly2), the rest to MUFU ex2: the two units share the load
+                // (exp2_sat_poly2 / exp2_poly2), the rest to MUFU ex2: the two
+                // units share the load
 #pragma unroll
                 for (int c = 0; c < BLK / 2; c += 4) {
 #pragma unroll
@@ -513,7 +531,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                         else a0 = fadd2(a0, xv[c + u]);
                     }
                 }
-                sum = (a0.x + a0.y) + (a1.x + a1.y);
+                sum = ((a0.x + a0.y) + (a1.x + a1.y)) * inv_fv;
             }
             l = l * alpha + sum;
             // P_X -> TMEM over S_X

@@ -56,6 +56,10 @@ struct KParams {
     // (test-only; 0 in every normal call)
     int withhold_k_item;
     int attn_kernel;           // 0: two-tile kernel, 1: one-tile kernel
+    // e4m3 only, optional: per-block scale factors in (0, 1] of K and V,
+    // [S][nkb_max][Hkv] (x = e4m3 * k_scale[h] * factor), or nullptr
+    const float* kb_fac;
+    const float* vb_fac;
 };
 
 // Detail codes stored beside an error code.
@@ -63,6 +67,7 @@ enum : uint32_t {
     kDetSeqLen = 1,      // Lq or Lk outside [0, max_seqlen_*] or Lk < Lq
     kDetPage = 3,        // page id outside [0, num_pages)
     kDetSlot = 4,        // block-mean cache slot outside [0, num_slots) or beyond max_blocks
+    kDetFactor = 5,      // a per-block scale factor outside (0, 1]
     kDetWaitBase = 16,   // + pipeline wait site
 };
 

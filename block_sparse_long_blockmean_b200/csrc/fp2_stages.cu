@@ -38,36 +38,80 @@ __device__ __forceinline__ void unpack16(const uint4& v, float* out) {
 }
 
 // ------------------------------------------------------------- blockmean ---
-// grid (nkb_max, Hkv, num_seqs), 128 threads.  Each CTA averages the valid
-// rows of one key block of one KV head, for K and V.  Blocks past the end
-// of the sequence are written as zeros (the attention kernel reads whole
-// tiles of means and multiplies the unused ones by zero).
-template <int D, bool FP8>
-__global__ void __launch_bounds__(128) blockmean_kernel(KParams p, const uint8_t* __restrict__ K,
-                                                        const uint8_t* __restrict__ V) {
-    constexpr int ELT = FP8 ? 1 : 2;
-    constexpr int VEC = 16 / ELT;   // elements per 16-byte load
-    constexpr int TPR = D / VEC;    // threads per row
-    constexpr int RPP = 128 / TPR;  // rows per pass
-    __shared__ float red[2][RPP][D];
+// grid (kb_n, num_seqs, ceil(Hkv*d / 1024)), 256 threads, one CTA per key
+// block of one sequence and slice of at most 1024 of the Hkv*d columns (all
+// KV heads when Hkv*d <= 1024).  The block's rows are contiguous in the cache
+// (within a page, for a paged one), so they stream through shared memory by
+// untiled bulk copies -- R rows of K and R of V per stage, kBmStages stages in
+// flight -- while the threads add up the stage before: thread t owns columns
+// 4t..4t+3 of the slice.  Blocks past the end of the sequence are written as
+// zeros (the attention kernel reads whole tiles of means and multiplies the
+// unused ones by zero).
+constexpr int kBmThreads = 256, kBmStages = 3, kBmSlice = 4 * kBmThreads;
+constexpr uint64_t kBmWaitNs = 2000000000ull;  // 2 s per stage wait
 
-    const int j = p.kb_lo + (int)blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+// rows per stage: at most 16 (they then never cross a page of >= 16 tokens)
+// and at most 16 KB of one tensor
+__host__ __device__ constexpr int bm_rows(int slice_bytes) {
+    return slice_bytes <= 1024 ? 16 : (slice_bytes <= 2048 ? 8 : 4);
+}
+
+template <bool FP8>
+__device__ __forceinline__ void unpack4(const uint8_t* src, float* out) {
+    if constexpr (FP8) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+            __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w >> (8 * e)) & 0xFFFFu);
+            __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+            float2 f = __half22float2(*reinterpret_cast<__half2*>(&h));
+            out[e] = f.x;
+            out[e + 1] = f.y;
+        }
+    } else {
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        out[0] = __uint_as_float(w.x << 16);
+        out[1] = __uint_as_float(w.x & 0xFFFF0000u);
+        out[2] = __uint_as_float(w.y << 16);
+        out[3] = __uint_as_float(w.y & 0xFFFF0000u);
+    }
+}
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(kBmThreads) blockmean_kernel(KParams p, const uint8_t* __restrict__ K,
+                                                               const uint8_t* __restrict__ V) {
+    constexpr int ELT = FP8 ? 1 : 2;
+    extern __shared__ __align__(128) uint8_t bm_smem[];
+    const int j = p.kb_lo + (int)blockIdx.x, b = blockIdx.y;
+    const int W = p.Hkv * D;                               // columns of a row
+    const int c0 = (int)blockIdx.z * kBmSlice;             // this CTA's columns
+    const int WS = min(kBmSlice, W - c0);
+    const size_t row_bytes = (size_t)W * ELT;
+    const int R = bm_rows(WS * ELT);
+    const int g = threadIdx.x, col = c0 + 4 * g;           // first of this thread's 4 columns
+    const bool has_col = 4 * g < WS;
+
     SeqInfo s;
     if (!load_seq(p, b, s)) return;
     const int nkb = (s.Lk + p.B - 1) / p.B;
-    const size_t orow = (((size_t)b * p.Hkv + hk) * p.nkb_max + j) * D;
+    auto out_at = [&](int c) {  // [S][Hkv][nkb_max][d] index of column c of block j
+        return (((size_t)b * p.Hkv + c / D) * p.nkb_max + j) * D + (c % D);
+    };
     if (j >= nkb) {
-        for (int c = threadIdx.x; c < D; c += 128) {
-            p.kbar[orow + c] = 0.f;
-            p.vbar[orow + c] = 0.f;
-            if constexpr (FP8) {
-                reinterpret_cast<uint8_t*>(p.kbar_op)[orow + c] = 0;
-                reinterpret_cast<uint8_t*>(p.vbar_op)[orow + c] = 0;
-            } else {
-                reinterpret_cast<__nv_bfloat16*>(p.kbar_op)[orow + c] = __float2bfloat16(0.f);
-                reinterpret_cast<__nv_bfloat16*>(p.vbar_op)[orow + c] = __float2bfloat16(0.f);
+        if (has_col)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const size_t o = out_at(col + e);
+                p.kbar[o] = 0.f;
+                p.vbar[o] = 0.f;
+                if constexpr (FP8) {
+                    reinterpret_cast<uint8_t*>(p.kbar_op)[o] = 0;
+                    reinterpret_cast<uint8_t*>(p.vbar_op)[o] = 0;
+                } else {
+                    reinterpret_cast<__nv_bfloat16*>(p.kbar_op)[o] = __float2bfloat16(0.f);
+                    reinterpret_cast<__nv_bfloat16*>(p.vbar_op)[o] = __float2bfloat16(0.f);
+                }
             }
-        }
         return;
     }
     const int t0 = j * p.B;
@@ -81,64 +125,130 @@ __global__ void __launch_bounds__(128) blockmean_kernel(KParams p, const uint8_t
             set_error(p.err, kErrBounds, kDetSlot);
             return;
         }
-        slot_ptr = p.mean_cache + ((size_t)slot * 2 * p.Hkv + hk) * D;
+        slot_ptr = p.mean_cache + (size_t)slot * 2 * W;
     }
-    const float ks = FP8 ? p.k_scale[hk] : 1.f;
-    const float vs = FP8 ? p.v_scale[hk] : 1.f;
+    // per-block scale factors (e4m3 caches quantised per key block): the
+    // means are dequantised with the block's scale and handed to the MMA in
+    // units of the per-head scale, the unit of every mean tile
     auto emit = [&](int c, float mk, float mv) {  // mk, mv: means of the stored values
-        p.kbar[orow + c] = mk * ks;                // dequantised
-        p.vbar[orow + c] = mv * vs;
+        const int hk = c / D;
+        float fk = 1.f, fv = 1.f;
         if constexpr (FP8) {
-            reinterpret_cast<__nv_fp8_e4m3*>(p.kbar_op)[orow + c] = __nv_fp8_e4m3(mk);
-            reinterpret_cast<__nv_fp8_e4m3*>(p.vbar_op)[orow + c] = __nv_fp8_e4m3(mv);
+            if (p.kb_fac) {
+                const size_t fi = ((size_t)b * p.nkb_max + j) * p.Hkv + hk;
+                fk = p.kb_fac[fi];
+                fv = p.vb_fac[fi];
+                if (!(fk > 0.f && fk <= 1.f && fv > 0.f && fv <= 1.f)) {
+                    set_error(p.err, kErrInvalid, kDetFactor);
+                    fk = fv = 1.f;
+                }
+            }
+        }
+        const size_t o = out_at(c);
+        p.kbar[o] = mk * (FP8 ? p.k_scale[hk] * fk : 1.f);  // dequantised
+        p.vbar[o] = mv * (FP8 ? p.v_scale[hk] * fv : 1.f);
+        if constexpr (FP8) {
+            reinterpret_cast<__nv_fp8_e4m3*>(p.kbar_op)[o] = __nv_fp8_e4m3(mk * fk);
+            reinterpret_cast<__nv_fp8_e4m3*>(p.vbar_op)[o] = __nv_fp8_e4m3(mv * fv);
         } else {
-            reinterpret_cast<__nv_bfloat16*>(p.kbar_op)[orow + c] = __float2bfloat16(mk);
-            reinterpret_cast<__nv_bfloat16*>(p.vbar_op)[orow + c] = __float2bfloat16(mv);
+            reinterpret_cast<__nv_bfloat16*>(p.kbar_op)[o] = __float2bfloat16(mk);
+            reinterpret_cast<__nv_bfloat16*>(p.vbar_op)[o] = __float2bfloat16(mv);
         }
     };
     if (slot_ptr && t0 + p.B <= s.P) {
-        for (int c = threadIdx.x; c < D; c += 128)
-            emit(c, slot_ptr[c], slot_ptr[(size_t)p.Hkv * D + c]);
+        if (has_col)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) emit(col + e, slot_ptr[col + e], slot_ptr[W + col + e]);
         return;
     }
-    const int lv = threadIdx.x % TPR, rg = threadIdx.x / TPR;
-    float ak[VEC], av[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) ak[e] = av[e] = 0.f;
-    for (int r = rg; r < n; r += RPP) {
-        const long long row = key_row(p, s, b, t0 + r);
-        if (row < 0) continue;
-        const size_t off = ((size_t)row * p.Hkv + hk) * D * ELT + (size_t)lv * 16;
-        const uint4 kv = __ldg(reinterpret_cast<const uint4*>(K + off));
-        const uint4 vv = __ldg(reinterpret_cast<const uint4*>(V + off));
-        float fk[VEC], fv[VEC];
-        unpack16<FP8>(kv, fk);
-        unpack16<FP8>(vv, fv);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            ak[e] += fk[e];
-            av[e] += fv[e];
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-        red[0][rg][lv * VEC + e] = ak[e];
-        red[1][rg][lv * VEC + e] = av[e];
+
+    // the ring: kBmStages barriers, then per stage R rows of K and R of V
+    uint64_t* bars = reinterpret_cast<uint64_t*>(bm_smem);
+    int* stage_rows = reinterpret_cast<int*>(bm_smem + 64);   // rows the stage holds
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bm_smem + 96);
+    uint8_t* ring = bm_smem + 128;
+    const size_t tile = (size_t)R * WS * ELT;                 // one tensor's rows of a stage
+    const bool whole_rows = WS == W;                          // one copy per tensor and stage
+    const int nst = (n + R - 1) / R;
+    if (threadIdx.x == 0) {
+        for (int k = 0; k < kBmStages; ++k) mbar_init(&bars[k], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
     }
     __syncthreads();
-    const float inv = 1.f / (float)n;
-    for (int c = threadIdx.x; c < D; c += 128) {
-        float sk = 0.f, sv = 0.f;
-#pragma unroll
-        for (int r = 0; r < RPP; ++r) {
-            sk += red[0][r][c];
-            sv += red[1][r][c];
+    // thread 0: stage st into slot st % kBmStages (rows of one page, or of the
+    // contiguous cache)
+    auto issue = [&](int st) {
+        const int slot = st % kBmStages, r0 = st * R, nr = min(R, n - r0);
+        const long long row = key_row(p, s, b, t0 + r0);
+        uint64_t* bar = &bars[slot];
+        stage_rows[slot] = row >= 0 ? nr : 0;
+        const uint32_t dst = smem_u32(ring + slot * 2 * tile);
+        if (row < 0) {
+            mbar_arrive(bar);
+        } else if (whole_rows) {
+            const uint32_t bytes = (uint32_t)(nr * row_bytes);
+            mbar_arrive_expect_tx(bar, 2 * bytes);
+            bulk_load(dst, K + row * row_bytes, bytes, bar);
+            bulk_load(dst + tile, V + row * row_bytes, bytes, bar);
+        } else {
+            const uint32_t bytes = (uint32_t)(WS * ELT);
+            mbar_arrive_expect_tx(bar, 2 * bytes * nr);
+            for (int r = 0; r < nr; ++r) {
+                const size_t src = (row + r) * row_bytes + (size_t)c0 * ELT;
+                bulk_load(dst + r * bytes, K + src, bytes, bar);
+                bulk_load(dst + tile + r * bytes, V + src, bytes, bar);
+            }
         }
-        const float mk = sk * inv, mv = sv * inv;
-        emit(c, mk, mv);
-        if (slot_ptr) {
-            slot_ptr[c] = mk;
-            slot_ptr[(size_t)p.Hkv * D + c] = mv;
+    };
+    if (threadIdx.x == 0)
+        for (int st = 0; st < min(kBmStages - 1, nst); ++st) issue(st);
+    float ak[4] = {0.f, 0.f, 0.f, 0.f}, av[4] = {0.f, 0.f, 0.f, 0.f};
+    int issued = min(kBmStages - 1, nst), done = 0;
+    for (int st = 0; st < nst; ++st) {
+        if (threadIdx.x == 0 && issued < nst) issue(issued++);
+        const bool ok = mbar_wait(&bars[st % kBmStages], (st / kBmStages) & 1, abort_flag, kBmWaitNs);
+        if (__syncthreads_or(!ok)) {
+            if (threadIdx.x == 0) set_error(p.err, kErrTimeout, kDetWaitBase + 13);
+            break;
+        }
+        const int slot = st % kBmStages, nr = stage_rows[slot];
+        if (has_col) {
+            const uint8_t* kt = ring + slot * 2 * tile + (size_t)4 * g * ELT;
+            for (int r = 0; r < nr; ++r) {
+                float fk[4], fv[4];
+                unpack4<FP8>(kt + (size_t)r * WS * ELT, fk);
+                unpack4<FP8>(kt + tile + (size_t)r * WS * ELT, fv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    ak[e] += fk[e];
+                    av[e] += fv[e];
+                }
+            }
+        }
+        done = st + 1;
+        __syncthreads();  // the slot may be refilled
+    }
+    if (done < nst) {
+        // aborted: let the copies already issued land before the CTA ends
+        if (threadIdx.x == 0) {
+            volatile int no_abort = 0;
+            for (int st = done; st < issued; ++st)
+                mbar_wait(&bars[st % kBmStages], (st / kBmStages) & 1, &no_abort, kBmWaitNs);
+        }
+        __syncthreads();
+        return;
+    }
+    if (has_col) {
+        const float inv = 1.f / (float)n;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float mk = ak[e] * inv, mv = av[e] * inv;
+            emit(col + e, mk, mv);
+            if (slot_ptr) {
+                slot_ptr[col + e] = mk;
+                slot_ptr[W + col + e] = mv;
+            }
         }
     }
 }
@@ -346,18 +456,28 @@ __global__ void __launch_bounds__(128) mask_kernel(KParams p, float tau) {
 
 // -------------------------------------------------------------- launchers ---
 cudaError_t launch_blockmean(const KParams& p, const void* k, const void* v, cudaStream_t st) {
-    dim3 grid(p.kb_n, p.Hkv, p.num_seqs);
     if (p.kb_n <= 0) return cudaSuccess;
+    const int W = p.Hkv * p.d;
+    if (W % 4 != 0) return cudaErrorInvalidValue;
+    const int elt = p.fp8 ? 1 : 2;
+    const int WS = W < kBmSlice ? W : kBmSlice;
+    const size_t smem = 128 + (size_t)kBmStages * 2 * bm_rows(WS * elt) * WS * elt;
+    dim3 grid(p.kb_n, p.num_seqs, (W + kBmSlice - 1) / kBmSlice);
     auto K = static_cast<const uint8_t*>(k);
     auto V = static_cast<const uint8_t*>(v);
+    cudaError_t e = cudaSuccess;
+    auto go = [&](auto kern) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess) kern<<<grid, kBmThreads, smem, st>>>(p, K, V);
+    };
     if (p.fp8) {
-        if (p.d == 128) blockmean_kernel<128, true><<<grid, 128, 0, st>>>(p, K, V);
-        else blockmean_kernel<64, true><<<grid, 128, 0, st>>>(p, K, V);
+        if (p.d == 128) go(blockmean_kernel<128, true>);
+        else go(blockmean_kernel<64, true>);
     } else {
-        if (p.d == 128) blockmean_kernel<128, false><<<grid, 128, 0, st>>>(p, K, V);
-        else blockmean_kernel<64, false><<<grid, 128, 0, st>>>(p, K, V);
+        if (p.d == 128) go(blockmean_kernel<128, false>);
+        else go(blockmean_kernel<64, false>);
     }
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D, bool FP8>

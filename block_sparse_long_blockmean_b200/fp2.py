@@ -62,6 +62,8 @@ class Params(ctypes.Structure):
         ("attn_kernel", ctypes.c_int),
         ("debug_wait_limit_us", ctypes.c_uint),
         ("debug_withhold_k_item", ctypes.c_int),
+        ("k_block_factor", ctypes.c_void_p),
+        ("v_block_factor", ctypes.c_void_p),
     ]
 
 
@@ -349,7 +351,8 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
                  page_table=None, page_size: int = 0, q_scale=None, k_scale=None,
                  v_scale=None, out=None, stream=None, workspace=None,
                  group_masks: bool = False, out_dtype: int = FP2_BF16,
-                 out_scale=None, attn_kernel: int = 0) -> Problem:
+                 out_scale=None, attn_kernel: int = 0, k_block_factor=None,
+                 v_block_factor=None) -> Problem:
     """Builds fp2_params for device tensors and allocates the workspace and
     the bf16 output with torch (allocation only)."""
     import torch
@@ -373,6 +376,8 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
     P.out_dtype = out_dtype
     P.out_scale = _ptr(out_scale)
     P.attn_kernel = int(attn_kernel)
+    P.k_block_factor = _ptr(k_block_factor)
+    P.v_block_factor = _ptr(v_block_factor)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
     P.stream = stream
@@ -387,5 +392,6 @@ def make_problem(q, k, v, cu_seqlens, *, Hq: int, Hkv: int, d: int, block: int, 
     if out is None:
         odt = torch.float8_e4m3fn if out_dtype == FP2_FP8_E4M3 else torch.bfloat16
         out = torch.empty((q.shape[0], Hq, d), dtype=odt, device=dev)
-    keep = (seqlens_k, cu_seqlens_k, q_scale, k_scale, v_scale, out_scale)
+    keep = (seqlens_k, cu_seqlens_k, q_scale, k_scale, v_scale, out_scale, k_block_factor,
+            v_block_factor)
     return Problem(q, k, v, page_table, cu_seqlens, out, block, dtype, P, workspace, keep)

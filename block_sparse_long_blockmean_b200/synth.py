@@ -21,7 +21,12 @@ makes max-based block selection meaningful):
   (saturating, round to nearest even);
 * paged caches: ``page_size`` tokens per page, pages of every sequence drawn
   from one seeded random permutation of all pages; unused page-table entries
-  are -1.
+  are -1;
+* ``kv_scales="block"`` (e4m3 only): the V rows of key block j of KV head h
+  are drawn times 2^(-3 u), u ~ U[0, 1) per (sequence, block, head), so that
+  blocks differ in magnitude, and K and V are quantised with one scale per
+  (sequence, key block, KV head), absmax/448; each is given as a factor in
+  (0, 1] of the per-head reference scale, the largest block scale of the head.
 """
 from __future__ import annotations
 
@@ -47,6 +52,7 @@ class Shape:
     page_size: int = 0           # 0 = contiguous K/V
     drop: float = 0.8            # target dropped fraction of causal block pairs
     seed: int = 20260822
+    kv_scales: str = "head"      # "head" | "block" (e4m3: one K/V scale per key block)
 
 
 # The five workloads (sizes from the FlashPrefill V2 setting: 128K context on
@@ -97,6 +103,10 @@ class Inputs:
     v_scale: torch.Tensor | None
     _kc: torch.Tensor = field(repr=False, default=None)  # contiguous K (quantised)
     _vc: torch.Tensor = field(repr=False, default=None)
+    # per-block scale factors [S, nkb_max, Hkv] (x = e4m3 * scale[h] * factor),
+    # or None (one scale per head)
+    k_block_factor: torch.Tensor | None = None
+    v_block_factor: torch.Tensor | None = None
 
     @property
     def num_seqs(self) -> int:
@@ -117,13 +127,20 @@ class Inputs:
         a, e = int(self.cu_seqlens_q[b]), int(self.cu_seqlens_q[b + 1])
         return self._deq(self.q[a:e], self.q_scale)
 
+    def _deq_kv(self, x: torch.Tensor, scale, factor, b: int) -> np.ndarray:
+        y = self._deq(x, scale)
+        if factor is not None:
+            rows = np.arange(y.shape[0]) // self.shape.B  # key block of each row
+            y = y * factor[b].to(torch.float64).numpy()[rows][:, :, None]
+        return y
+
     def seq_k(self, b: int) -> np.ndarray:
         a, e = int(self.cu_seqlens_k[b]), int(self.cu_seqlens_k[b + 1])
-        return self._deq(self._kc[a:e], self.k_scale)
+        return self._deq_kv(self._kc[a:e], self.k_scale, self.k_block_factor, b)
 
     def seq_v(self, b: int) -> np.ndarray:
         a, e = int(self.cu_seqlens_k[b]), int(self.cu_seqlens_k[b + 1])
-        return self._deq(self._vc[a:e], self.v_scale)
+        return self._deq_kv(self._vc[a:e], self.v_scale, self.v_block_factor, b)
 
     def seq_q_rows(self, b: int, rows: np.ndarray) -> np.ndarray:
         a = int(self.cu_seqlens_q[b])
@@ -141,6 +158,34 @@ def _quantise(x: np.ndarray, dtype: str):
         y = (t / scale[None, :, None]).clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
         return y, scale
     raise ValueError(dtype)
+
+
+def _quantise_blocks(parts: list, B: int):
+    """Per-block e4m3 quantisation of per-sequence fp32 [L, H, d] arrays:
+    (concatenated e4m3 tensor, per-head reference scale [H], factors
+    [S, nkb_max, H] in (0, 1]; unused entries 1)."""
+    H = parts[0].shape[1]
+    nkb = max(-(-p.shape[0] // B) for p in parts)
+    bscale = np.ones((len(parts), nkb, H), dtype=np.float64)
+    for b, x in enumerate(parts):
+        for j in range(-(-x.shape[0] // B)):
+            amax = np.abs(x[j * B:(j + 1) * B]).max(axis=(0, 2)).astype(np.float64)
+            bscale[b, j] = np.maximum(amax, 1e-12) / E4M3_MAX
+    ref = np.zeros(H)
+    for b, x in enumerate(parts):
+        n = -(-x.shape[0] // B)
+        ref = np.maximum(ref, bscale[b, :n].max(axis=0))
+    ref32 = ref.astype(np.float32)
+    fac = np.ones((len(parts), nkb, H), dtype=np.float32)
+    out = []
+    for b, x in enumerate(parts):
+        n = -(-x.shape[0] // B)
+        f = (bscale[b, :n] / ref).astype(np.float32)
+        fac[b, :n] = f
+        sc = (ref32[None, :] * f)[np.arange(x.shape[0]) // B]  # scale of each row [L, H]
+        y = torch.from_numpy(x / sc[:, :, None]).clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+        out.append(y)
+    return torch.cat(out, dim=0), torch.from_numpy(ref32), torch.from_numpy(fac)
 
 
 def make_inputs(s: Shape, layout: str | None = None) -> Inputs:
@@ -172,14 +217,27 @@ def make_inputs(s: Shape, layout: str | None = None) -> Inputs:
         qn += 1.5 * c[head_kv[None, :], zq[:, None], :]
         kn += 1.5 * c[np.arange(Hkv)[None, :], zk[:, None], :]
         kn[:4] *= 3.0
+        if s.kv_scales == "block":
+            vv *= np.exp2(-3.0 * rng.random((nblk, Hkv), dtype=np.float32))[np.arange(Lk) // B][:, :, None]
         qs.append(qn); ks.append(kn); vs.append(vv)
-    qf = np.concatenate(qs, axis=0)
-    kf = np.concatenate(ks, axis=0)
-    vf = np.concatenate(vs, axis=0)
-    del qs, ks, vs
-    q, q_scale = _quantise(qf, s.dtype); del qf
-    kc, k_scale = _quantise(kf, s.dtype); del kf
-    vc, v_scale = _quantise(vf, s.dtype); del vf
+    kfac = vfac = None
+    if s.kv_scales == "block":
+        if s.dtype != "fp8":
+            raise ValueError("per-block scales are an e4m3 input format")
+        kc, k_scale, kfac = _quantise_blocks(ks, B)
+        vc, v_scale, vfac = _quantise_blocks(vs, B)
+        del ks, vs
+        qf = np.concatenate(qs, axis=0)
+        del qs
+        q, q_scale = _quantise(qf, s.dtype); del qf
+    else:
+        qf = np.concatenate(qs, axis=0)
+        kf = np.concatenate(ks, axis=0)
+        vf = np.concatenate(vs, axis=0)
+        del qs, ks, vs
+        q, q_scale = _quantise(qf, s.dtype); del qf
+        kc, k_scale = _quantise(kf, s.dtype); del kf
+        vc, v_scale = _quantise(vf, s.dtype); del vf
     cu_q = torch.tensor(np.concatenate([[0], np.cumsum(s.lens_q)]), dtype=torch.int32)
     cu_k = torch.tensor(np.concatenate([[0], np.cumsum(s.lens_k)]), dtype=torch.int32)
     seqlens_k = torch.tensor(s.lens_k, dtype=torch.int32)
@@ -187,7 +245,7 @@ def make_inputs(s: Shape, layout: str | None = None) -> Inputs:
     layout = layout or ("paged" if s.page_size else "contiguous")
     if layout == "contiguous":
         return Inputs(s, q, kc, vc, cu_q, cu_k, seqlens_k, None, q_scale, k_scale, v_scale,
-                      kc, vc)
+                      kc, vc, kfac, vfac)
     ps = s.page_size or 64
     npages = [-(-int(L) // ps) for L in s.lens_k]
     total_pages = int(sum(npages))
@@ -213,4 +271,4 @@ def make_inputs(s: Shape, layout: str | None = None) -> Inputs:
             vcache[phys, :n] = vc[a + p * ps: a + p * ps + n]
         off += npages[b]
     return Inputs(s, q, kcache, vcache, cu_q, cu_k, seqlens_k, torch.from_numpy(table),
-                  q_scale, k_scale, v_scale, kc, vc)
+                  q_scale, k_scale, v_scale, kc, vc, kfac, vfac)

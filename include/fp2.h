@@ -122,6 +122,16 @@ typedef struct fp2_params {
                                   (1-based) in any CTA, so the consumer's bounded wait runs
                                   out and the call records FP2_ERR_TIMEOUT; the output is
                                   then undefined.  Never set in normal use */
+    const float* k_block_factor; /* e4m3 only, optional (NULL: one scale per head): a KV
+                                  cache quantised per key block.  Device fp32
+                                  [num_seqs][ceil(max_seqlen_k / block)][Hkv]: key block j of
+                                  sequence b, KV head h dequantises as
+                                  x = e4m3 * k_scale[h] * k_block_factor[b][j][h], factor in
+                                  (0, 1] (k_scale[h] is then the head's largest block scale).
+                                  A factor outside (0, 1] records FP2_ERR_INVALID_ARG
+                                  (detail 5) on the device.  Given together with
+                                  v_block_factor; the two-tile attention kernel only */
+    const float* v_block_factor; /* the same for V */
 } fp2_params;
 
 /* Offsets (bytes from params->workspace) of the intermediates, for callers

@@ -28,6 +28,8 @@ def problem(inp: synth.Inputs, dev: str = "cuda", out_fill: float | None = None,
     pt = inp.page_table.to(dev) if inp.paged else None
     cu_k = None if inp.paged else inp.cu_seqlens_k.to(dev)
     sc = [x.to(dev) if x is not None else None for x in (inp.q_scale, inp.k_scale, inp.v_scale)]
+    fac = [x.contiguous().to(dev) if x is not None else None
+           for x in (inp.k_block_factor, inp.v_block_factor)]
     out = None
     if out_fill is not None:
         out = torch.full((q.shape[0], s.Hq, s.d), out_fill, dtype=torch.bfloat16, device=dev)
@@ -36,7 +38,8 @@ def problem(inp: synth.Inputs, dev: str = "cuda", out_fill: float | None = None,
                           seqlens_k=lk, cu_seqlens_k=cu_k, page_table=pt,
                           page_size=s.page_size or (k.shape[1] if inp.paged else 0),
                           q_scale=sc[0], k_scale=sc[1], v_scale=sc[2], out=out,
-                          group_masks=group_masks, attn_kernel=attn_kernel)
+                          group_masks=group_masks, attn_kernel=attn_kernel,
+                          k_block_factor=fac[0], v_block_factor=fac[1])
     if ws_fill is not None:
         pr.workspace.fill_(ws_fill)
         fp2.workspace_init(pr.params)
@@ -143,9 +146,10 @@ def oracle_out(inp: synth.Inputs, b: int, orc_b, keep, rows=None, heads=None):
 
 
 def small_shape(lens_q, lens_k=None, Hq=8, Hkv=2, d=128, B=128, dtype="bf16", page_size=0,
-                drop=0.7, seed=7, latents="shared16") -> synth.Shape:
+                drop=0.7, seed=7, latents="shared16", kv_scales="head") -> synth.Shape:
     lens_k = list(lens_q) if lens_k is None else list(lens_k)
-    return synth.Shape(list(lens_q), lens_k, Hq, Hkv, d, B, dtype, latents, page_size, drop, seed)
+    return synth.Shape(list(lens_q), lens_k, Hq, Hkv, d, B, dtype, latents, page_size, drop, seed,
+                       kv_scales)
 
 
 def drop_fraction(keeps, orc) -> float:
