@@ -21,9 +21,10 @@
 // 224 per softmax thread, 56 in the control warpgroup, 384 x 168 in total):
 //   warps 0-3  softmax for tile A (thread = row = TMEM lane)
 //   warps 4-7  softmax for tile B
-//   warp 8     TMA producer of the K and V rings (2 stages each; the two Q
-//              tiles are fetched by thread 0 right after the barriers exist)
-//   warps 10-11 idle
+//   warp 8     TMA producer of the K ring, warp 10 of the V ring (2 stages
+//              each; the two Q tiles are fetched by thread 0 right after the
+//              barriers exist)
+//   warp 11    idle
 //   warp 9     TMEM owner; lane 0 issues the MMAs in the order
 //                PV_A(n-1), QK_A(n), PV_B(n-1), QK_B(n)
 //              so that while one warpgroup works on its S the tensor core
@@ -58,40 +59,26 @@ struct PairCfg {
     static constexpr int OFF_RING = OFF_MISC + 64;  // page ids of upcoming items
     static constexpr int OFF_ITEMS = OFF_RING + 2 * kPageRing * kMaxBoxes * 4;  // K and V rings
     static_assert(P_COLS % 32 == 0, "P row must be whole 32-column TMEM stores");
-    // pairs (of every 4) whose exp2 runs on the FMA pipe: the fp8 MMA is twice
-    // as fast, so more of the exp2 work moves off the MUFU unit there
-#ifndef FP2_EMU_PAIRS_FP8
-#define FP2_EMU_PAIRS_FP8 1
-#endif
-#ifndef FP2_EMU_PAIRS_BF16
-#define FP2_EMU_PAIRS_BF16 1
-#endif
-    static constexpr int kEmuPairs = FP8 ? FP2_EMU_PAIRS_FP8 : FP2_EMU_PAIRS_BF16;
+    // pairs (of every 4) whose exp2 runs on the FMA pipe instead of MUFU (one
+    // measured best for both types; 0, 2 and 3 were slower)
+    static constexpr int kEmuPairs = 1;
     // polynomial degree of the FMA-pipe exp2: e4m3 probabilities need less
-#ifndef FP2_EMU_DEG_FP8
-#define FP2_EMU_DEG_FP8 2
-#endif
-    static constexpr int kEmuDeg = FP8 ? FP2_EMU_DEG_FP8 : 3;
+    static constexpr int kEmuDeg = FP8 ? 2 : 3;
 };
 
-// FMA-pipe exp2 with the clamp folded into a saturating FMA (exp2_sat_poly2)
-// instead of two fmax on the ALU pipe.  Its range ends at exponent 8, which
-// the lazy rescale guarantees: every exponent is x * sl2 + bias - m_used with
-// the row's maximum at most kRescaleLog2 above m_used.
-#ifndef FP2_EXP_SAT
-#define FP2_EXP_SAT 1
-#endif
-static_assert(!FP2_EXP_SAT || kRescaleLog2 <= 8.f, "exp2_sat_poly2 covers exponents up to 8");
+// The FMA-pipe exp2 (exp2_sat_poly2) folds its clamp into a saturating FMA;
+// its range ends at exponent 8, which the lazy rescale guarantees: every
+// exponent is x * sl2 + bias - m_used with the row's maximum at most
+// kRescaleLog2 above m_used.
+static_assert(kRescaleLog2 <= 8.f, "exp2_sat_poly2 covers exponents up to 8");
 
-#ifndef FP2_SPLIT_PRODUCER
-#define FP2_SPLIT_PRODUCER 1
-#endif
 
 // K and V have separate rings: K(n) is free once QK_B(n) has run, V(n) only
 // after PV_B(n) -- a full MMA pair later -- so each stream refills as soon as
 // its own operand is consumed.
-// KV_FULL[n % 2]: the producer's step n has landed, K(n) and V(n-1) together
-// (one barrier, so the MMA thread polls once per item for both)
+// KV_FULL[n % 2]: step n has landed, K(n) and V(n-1) together (one barrier
+// with one arrival per producer warp, so the MMA thread polls once per item
+// for both)
 enum { PB_KV_FULL = 0, PB_K_EMPTY = 2, PB_V_EMPTY = 4, PB_Q_FULL = 6, PB_S_FULL = 7,
        PB_P_READY = 9, PB_O_FINAL = 11, PB_DRAIN = 13, PB_COUNT = 14 };
 
@@ -148,7 +135,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
     if (threadIdx.x == 0) {
         for (int k = 0; k < PB_COUNT; ++k)
             mbar_init(&bars[k], (k == PB_P_READY || k == PB_P_READY + 1) ? 128u
-                                : (FP2_SPLIT_PRODUCER && k < PB_K_EMPTY) ? 2u : 1u);
+                                : k < PB_K_EMPTY ? 2u : 1u);  // KV_FULL: one arrival per producer
         misc[1] = 0;
         fence_mbar_init();
         // both Q tiles right away: their latency overlaps the kept-bit loads
@@ -179,7 +166,6 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     if (warp >= 8) {
       regs_decrease<56>();
-#if FP2_SPLIT_PRODUCER
       if (warp == 8 || warp == 10) {
         // --------------------------------------------------------- producers ---
         // warp 8 issues the K ring, warp 10 the V ring; each warp resolves
@@ -251,68 +237,6 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             if (is_k) drained &= mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, wlim);
             if (!drained) set_error(p.err, kErrTimeout, kDetWaitBase + 12);
         }
-#else
-      if (warp == 8) {
-        // ---------------------------------------------------------- producer ---
-        // the whole warp resolves page ids 32 items at a time; lane 0 waits
-        // and issues every copy
-        int* pring = reinterpret_cast<int*>(smem + C::OFF_RING);
-        if (lane == 0) {
-            prefetch_tmap(&maps.k);
-            prefetch_tmap(&maps.v);
-        }
-        // K runs one item ahead of V: step n loads K(n) and V(n-1), both
-        // counted on KV_FULL[n % 2] (K adds its bytes, V or a lone K arrives)
-        int steps = 0;  // 1 + the last producer step that issued a copy
-        bool ok = true;
-        for (int n = 0; n <= n_items; ++n) {
-            if (n % 32 == 0 && n < n_items) fill_page_ring<BLK>(p, s, b, items, n_items, n, pring);
-            if (lane == 0) {
-                uint64_t* full = &bars[PB_KV_FULL + n % C::S];
-                bool k_issued = false;
-                if (n < n_items) {
-                    const int st = n % C::S;
-                    if (n >= C::S && !mbar_wait(&bars[PB_K_EMPTY + st], ((n - C::S) / C::S) & 1,
-                                                abort_flag, wlim)) {
-                        set_error(p.err, kErrTimeout, kDetWaitBase + 0);
-                        ok = false;
-                    } else {
-                        issue_tile_load<D, BLK, FP8>(p, &maps.k, &maps.kb, s, b, hk, items[n],
-                                                     pring + (n % kPageRing) * kMaxBoxes,
-                                                     sbase + C::OFF_K + st * C::KV_BYTES, full,
-                                                     n == 0);
-                        k_issued = true;
-                        steps = n + 1;
-                    }
-                }
-                if (ok && n >= 1) {
-                    const int m = n - 1, st = m % C::S;
-                    if (m >= C::S && !mbar_wait(&bars[PB_V_EMPTY + st], ((m - C::S) / C::S) & 1,
-                                                abort_flag, wlim)) {
-                        set_error(p.err, kErrTimeout, kDetWaitBase + 0);
-                        ok = false;
-                        // K(n) went without an arrival: arrive so that the
-                        // step completes once its bytes land (drained below)
-                        if (k_issued) mbar_arrive(full);
-                    } else {
-                        issue_tile_load<D, BLK, FP8>(p, &maps.v, &maps.vb, s, b, hk, items[m],
-                                                     pring + (m % kPageRing) * kMaxBoxes,
-                                                     sbase + C::OFF_V + st * C::KV_BYTES, full,
-                                                     true);
-                        steps = n + 1;
-                    }
-                }
-            }
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        }
-        if (lane == 0) {
-            // never leave with copies in flight: the last steps that issued any
-            volatile int no_abort = 0;
-            for (int n = max(0, steps - C::S); n < steps; ++n)
-                mbar_wait(&bars[PB_KV_FULL + n % C::S], (n / C::S) & 1, &no_abort, wlim);
-            mbar_wait(&bars[PB_Q_FULL], 0, &no_abort, wlim);
-        }
-#endif
       } else if (warp == 9 && lane == 0) {
         // -------------------------------------------------------------- MMA ---
             constexpr uint32_t fmt = FP8 ? 0u : 1u;
@@ -511,18 +435,14 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
                 const float k128 = sl2i * (1.f / 128.f), c128 = (c0 + 120.f) * (1.f / 128.f);
                 float2 a0 = make_float2(0.f, 0.f), a1 = a0;
                 // of every 4 pairs, the last kEmuPairs go to the FMA pipe
-                // (exp2_sat_poly2 / exp2_poly2), the rest to MUFU ex2: the two
-                // units share the load
+                // (exp2_sat_poly2), the rest to MUFU ex2: the two units share
+                // the load
 #pragma unroll
                 for (int c = 0; c < BLK / 2; c += 4) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         if (u >= 4 - C::kEmuPairs) {
-#if FP2_EXP_SAT
                             xv[c + u] = exp2_sat_poly2<C::kEmuDeg>(xv[c + u], k128, c128);
-#else
-                            xv[c + u] = exp2_poly2<C::kEmuDeg>(ffma2(xv[c + u], k2, c2));
-#endif
                         } else {
                             const float2 e = ffma2(xv[c + u], k2, c2);
                             xv[c + u] = make_float2(ex2(e.x), ex2(e.y));

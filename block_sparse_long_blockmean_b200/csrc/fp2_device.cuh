@@ -315,36 +315,6 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
-// 2^x for a pair, on the FMA and integer pipes instead of the MUFU unit.
-// Cody-Waite reduction x = j + f (j = rint(x) by adding 1.5*2^23, exact for
-// |x| < 2^22), 2^f by a polynomial of fp2_exp2_poly.h -- degree 3 (relative
-// error < FP2_EXP2_REL_ERR on [-1/2, 1/2]) or degree 2 (< FP2_EXP2_Q_REL_ERR,
-// enough for values that are then rounded to e4m3) -- and 2^j added to the
-// exponent field.  Inputs are clamped to >= -126 so the exponent never
-// wraps: anything below (including -inf and NaN) returns a value <= 2^-125,
-// i.e. a zero weight.  Valid for x <= 127.
-template <int DEG>
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    static_assert(DEG == 2 || DEG == 3, "fitted degrees");
-    const float magic = 12582912.0f;  // 1.5 * 2^23
-    x.x = fmaxf(x.x, -126.0f);
-    x.y = fmaxf(x.y, -126.0f);
-    const float2 t = fadd2(x, make_float2(magic, magic));
-    const float2 j = fadd2(t, make_float2(-magic, -magic));
-    const float2 f = fadd2(x, make_float2(-j.x, -j.y));
-    float2 p;
-    if constexpr (DEG == 3) {
-        p = ffma2(f, make_float2(FP2_EXP2_C3, FP2_EXP2_C3), make_float2(FP2_EXP2_C2, FP2_EXP2_C2));
-        p = ffma2(p, f, make_float2(FP2_EXP2_C1, FP2_EXP2_C1));
-        p = ffma2(p, f, make_float2(FP2_EXP2_C0, FP2_EXP2_C0));
-    } else {
-        p = ffma2(f, make_float2(FP2_EXP2_Q2, FP2_EXP2_Q2), make_float2(FP2_EXP2_Q1, FP2_EXP2_Q1));
-        p = ffma2(p, f, make_float2(FP2_EXP2_Q0, FP2_EXP2_Q0));
-    }
-    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
     float d;
     asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -360,8 +330,13 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
     return d;
 }
 
-// 2^e for a pair with e = x * k + c, the clamp folded into the affine step
-// on the FMA pipe: y = sat(e / 128 + 120 / 128) maps e in [-120, 8] onto
+// 2^e for a pair, on the FMA and integer pipes instead of the MUFU unit,
+// with e = x * k + c.  Cody-Waite reduction e = j + f (j = rint(e) by adding
+// 1.5 * 2^23), 2^f by a polynomial of fp2_exp2_poly.h -- degree 3 (relative
+// error < FP2_EXP2_REL_ERR on [-1/2, 1/2]) or degree 2 (< FP2_EXP2_Q_REL_ERR,
+// enough for values that are then rounded to e4m3) -- and 2^j added to the
+// exponent field.  The clamp is folded into the affine step on the FMA pipe:
+// y = sat(e / 128 + 120 / 128) maps e in [-120, 8] onto
 // [0, 1] (saturating outside; -inf and NaN give 0), then
 //   t = y * 128 + (1.5 * 2^23 - 120) = 1.5 * 2^23 + j,  j = rint(e) (clamped)
 //   f = y * 128 - (j + 120) = e - j in [-1/2, 1/2]
