@@ -115,3 +115,23 @@ def test_single_stream_when_no_copy_streams_are_given():
     del keep
     assert torch.equal(out_host, ref.out.cpu())
     assert np.isfinite(out_host.float().numpy()).all()
+
+
+@pytest.mark.parametrize("page", [64, 0])
+def test_block_scaled_cache_through_host_path(page):
+    """An e4m3 cache quantised per key block (per-block factors stay device
+    arrays, like the lengths): the host path equals the device path bit for bit."""
+    kw = dict(lens_q=[700, 1, 300], lens_k=[700 + 256, 900, 300], Hq=8, Hkv=2, dtype="fp8",
+              page_size=page, kv_scales="block")
+    if not page:  # contiguous K/V carries no prefix
+        kw["lens_k"] = list(kw["lens_q"])
+    inp = synth.make_inputs(H.small_shape(**kw, seed=66))
+    tau = H.pick_tau(H.oracle_scores(inp), 0.6)
+    ref = device_reference(inp, tau)
+    pr = H.problem(inp, out_fill=float("nan"))
+    out_host = torch.full(pr.out.shape, float("nan"), dtype=pr.out.dtype).pin_memory()
+    keep = host_call(pr, inp, tau, 4, (torch.cuda.Stream(), torch.cuda.Stream()), out_host)
+    torch.cuda.synchronize()
+    pr.check()
+    del keep
+    assert torch.equal(out_host, ref.out.cpu())
