@@ -171,7 +171,7 @@ fp2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP2_OK : FP2_E
 // Events that order fp2_prefill_host's three streams: created once per device
 // on first use, re-recorded by every call while g_host_mutex is held (so a
 // record and the waits on it are never interleaved with another call's).
-constexpr int kHostMaxChunks = 16;
+constexpr int kHostMaxChunks = 64;
 constexpr int kHostEvents = 2 * kHostMaxChunks + 3;
 constexpr int kHostMaxDevices = 64;
 struct HostEvents {

@@ -265,7 +265,7 @@ typedef struct fp2_host_io {
                               params->stream (no overlap) */
     void* download_stream; /* cudaStream_t for the device->host copies; NULL:
                               params->stream (no overlap) */
-    int num_chunks;        /* query-block chunks of the pipeline, 1..16 */
+    int num_chunks;        /* query-block chunks of the pipeline, 1..64 */
 } fp2_host_io;
 
 /* fp2_prefill with q, K/V and out in host memory: the call a serving process
@@ -288,7 +288,7 @@ typedef struct fp2_host_io {
  *    first call (make it before any stream capture); calls from several
  *    host threads are serialised while they queue.
  *  - Errors as fp2_prefill; io == NULL, a NULL buffer, num_chunks outside
- *    [1, 16] or misaligned device buffers return FP2_ERR_INVALID_ARG. */
+ *    [1, 64] or misaligned device buffers return FP2_ERR_INVALID_ARG. */
 fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
                             const int32_t* cu_seqlens, float tau, int block, fp2_dtype dtype,
                             const fp2_params* params);

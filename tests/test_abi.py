@@ -230,7 +230,7 @@ def test_host_pipeline_rejects_bad_arguments_before_any_cuda_work(lib):
     for f, _ in fp2.HostIO._fields_:
         if f not in ("seqlens_k_host", "upload_stream", "download_stream", "num_chunks"):
             setattr(io, f, fake)
-    for chunks in (0, 17, -1):
+    for chunks in (0, 65, -1):
         io.num_chunks = chunks
         assert lib.fp2_prefill_host(ctypes.byref(io), None, fake, 1.0, 128, 0,
                                     ctypes.byref(P)) == fp2.FP2_ERR_INVALID_ARG

@@ -53,7 +53,7 @@ def host_call(pr, inp, tau, num_chunks, streams, out_host):
 
 
 @pytest.mark.parametrize("name", sorted(SHAPES))
-@pytest.mark.parametrize("num_chunks", [1, 3, 16])
+@pytest.mark.parametrize("num_chunks", [1, 3, 16, 64])
 def test_host_path_matches_device_path(name, num_chunks):
     inp = synth.make_inputs(H.small_shape(**SHAPES[name], seed=61))
     tau = H.pick_tau(H.oracle_scores(inp), 0.6)
