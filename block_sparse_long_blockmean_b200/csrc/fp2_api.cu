@@ -531,11 +531,17 @@ fp2_status fp2_prefill_host(const fp2_host_io* io, const int32_t* page_table,
         if (e == cudaSuccess) e = cudaMemsetAsync(kp.vbar_op, 0, op_bytes, s);
     }
     // query-block ranges, lowest first: a range needs the keys up to its last
-    // diagonal block, so the key upload grows with the ranges
-    const int per = (kp.nqb_max + io->num_chunks - 1) / io->num_chunks;
+    // diagonal block, so the key upload grows with the ranges.  Range c ends at
+    // nqb * ((c+1)/n)^0.7: causal work grows with the query position, so the
+    // early ranges are wider and the last ones, whose compute is the tail
+    // after the uploads, narrower (measured: 0.7 beats even ranges by about
+    // 1 % on the 128K layer; 0.6 does not)
+    auto bound = [&](int c) {
+        return (int)std::lround(kp.nqb_max * std::pow((double)c / io->num_chunks, 0.7));
+    };
     for (int c = 0; e == cudaSuccess && c < io->num_chunks; ++c) {
-        const int lo = c * per, hi = std::min(kp.nqb_max, lo + per);
-        if (lo >= hi) break;
+        const int lo = bound(c), hi = std::min(kp.nqb_max, bound(c + 1));
+        if (lo >= hi) continue;
         int kb_hi = kb_done;
         if (!paged) {
             for (int b = 0; b < S; ++b) kb_hi = std::max(kb_hi, pb[b] + hi);

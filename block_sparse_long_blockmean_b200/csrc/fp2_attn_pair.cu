@@ -134,7 +134,7 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
 
     if (threadIdx.x == 0) {
         for (int k = 0; k < PB_COUNT; ++k)
-            mbar_init(&bars[k], (k == PB_P_READY || k == PB_P_READY + 1) ? 128u
+            mbar_init(&bars[k], (k == PB_P_READY || k == PB_P_READY + 1) ? 4u  // one per softmax warp
                                 : k < PB_K_EMPTY ? 2u : 1u);  // KV_FULL: one arrival per producer
         misc[1] = 0;
         fence_mbar_init();
@@ -484,7 +484,8 @@ attn_pair_kernel(const KParams p, const __grid_constant__ AttnMaps maps,
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[PB_P_READY + X]);
+            __syncwarp();  // the warp's P stores (and V zeroing) before its one arrival
+            if (lane == 0) mbar_arrive(&bars[PB_P_READY + X]);
         }
         if (ok && __all_sync(0xffffffffu, mbar_wait(&bars[PB_O_FINAL + X], 0, abort_flag,
                                                     wlim))) {
