@@ -278,9 +278,9 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
     const int iabs = s.pb + i;
 
     const int v = threadIdx.x % VPT, tg = threadIdx.x / VPT;
-    float acc[VEC];
+    float2 acc[VEC / 2];  // packed adds: half the issue slots
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+    for (int e = 0; e < VEC / 2; ++e) acc[e] = make_float2(0.f, 0.f);
     const uint8_t* qrow = Q + (((size_t)(s.q0 + t0) * p.Hq + hk * G) * D) * ELT + (size_t)v * 16;
     const size_t tok_stride = (size_t)p.Hq * D * ELT;
     // 8 loads in flight per thread before any is consumed
@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
             float f[VEC];
             unpack16<FP8>(xs[u], f);
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) acc[e] += f[e];
+            for (int e = 0; e < VEC / 2; ++e) acc[e] = fadd2(acc[e], make_float2(f[2 * e], f[2 * e + 1]));
         }
     }
     for (; t < n; t += TPP) {
@@ -304,10 +304,13 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
         float f[VEC];
         unpack16<FP8>(x, f);
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] += f[e];
+        for (int e = 0; e < VEC / 2; ++e) acc[e] = fadd2(acc[e], make_float2(f[2 * e], f[2 * e + 1]));
     }
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) red[tg][v * VEC + e] = acc[e];
+    for (int e = 0; e < VEC / 2; ++e) {
+        red[tg][v * VEC + 2 * e] = acc[e].x;
+        red[tg][v * VEC + 2 * e + 1] = acc[e].y;
+    }
     __syncthreads();
     const float inv = 1.f / (float)n;
     for (int c = threadIdx.x; c < G * D; c += 256) {
@@ -343,74 +346,76 @@ __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int PER_LANE = D / 32;  // 4 (d=128) or 2 (d=64)
-    float qv[G][PER_LANE];
+    constexpr int NV = 4 * G;         // 4 key blocks x G heads per warp step: 4 .. 32 values
+    // Each warp takes 4 key blocks at a time: NV partial dot products per
+    // lane (lanes split d), summed over the warp by a reduce-scatter
+    // butterfly: the step with lane offset o (16, 8, ... while values remain)
+    // halves what a lane carries, lanes with bit o set keeping the upper half
+    // of the value indices.  So a lane ends up owning index m (below), and
+    // its value slot x holds the product for index x ^ m: then the half a
+    // lane keeps is always slots [0, half) and the half it sends [half, nv),
+    // and the partner's sent slot x + half is the same index as the kept
+    // slot x -- a shuffle and an add per value, no per-lane selects.
+    int m = 0;
+    {
+        int h = NV >> 1;
+#pragma unroll
+        for (int o = 16; o >= 1 && h >= 1; o >>= 1, h >>= 1)
+            if (lane & o) m += h;
+    }
+    const int m_r = m / G, m_g = m % G;  // index = key * G + head
+    // pooled queries in this lane's head order (slot g holds head g ^ m_g)
+    float2 qp[G][PER_LANE / 2];
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int e = 0; e < PER_LANE; ++e) qv[g][e] = qb[g * D + lane * PER_LANE + e];
+        for (int e = 0; e < PER_LANE / 2; ++e) {
+            const float* src = qb + (g ^ m_g) * D + lane * PER_LANE + 2 * e;
+            qp[g][e] = make_float2(src[0], src[1]);
+        }
     const float scale = rsqrtf((float)D);
     const float* kb = p.kbar + ((size_t)b * p.Hkv + hk) * p.nkb_max * D + lane * PER_LANE;
     float* srow = p.scores + (((size_t)b * p.Hq + hk * G) * p.nqb_max + i) * p.nkb_max;
     const size_t head_stride = (size_t)p.nqb_max * p.nkb_max;
-    // Each warp takes 4 key blocks at a time: 4*G partial dot products per
-    // lane (lanes split d), summed over the warp by a reduce-scatter
-    // butterfly (each step halves the values a lane carries), so that the
-    // 4*G sums end up spread over the lanes instead of every lane holding all.
-    constexpr int NV = 4 * G;  // 4, 8, 16 or 32 values
     for (int j0 = warp * 4; j0 <= iabs; j0 += 32) {
-        float v[NV];
+        float w[NV];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const int j = min(j0 + r, iabs);
-            float kv[PER_LANE];
+            // slot r*G + g: key block j0 + (r ^ m_r), head g ^ m_g
+            const int j = min(j0 + (r ^ m_r), iabs);
+            float2 kv[PER_LANE / 2];
             if constexpr (PER_LANE == 4) {
                 const float4 t4 = __ldg(reinterpret_cast<const float4*>(kb + (size_t)j * D));
-                kv[0] = t4.x; kv[1] = t4.y; kv[2] = t4.z; kv[3] = t4.w;
+                kv[0] = make_float2(t4.x, t4.y);
+                kv[1] = make_float2(t4.z, t4.w);
             } else {
-                const float2 t2 = __ldg(reinterpret_cast<const float2*>(kb + (size_t)j * D));
-                kv[0] = t2.x; kv[1] = t2.y;
+                kv[0] = __ldg(reinterpret_cast<const float2*>(kb + (size_t)j * D));
             }
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float a = 0.f;
+                float2 a = ffma2(qp[g][0], kv[0], make_float2(0.f, 0.f));
 #pragma unroll
-                for (int e = 0; e < PER_LANE; ++e) a = fmaf(qv[g][e], kv[e], a);
-                v[r * G + g] = a;
+                for (int e = 1; e < PER_LANE / 2; ++e) a = ffma2(qp[g][e], kv[e], a);
+                w[r * G + g] = a.x + a.y;
             }
         }
-        // reduce-scatter: after the step with offset o (o = 16, 8, ...), a lane
-        // keeps the half of its values selected by its bit o and adds the
-        // partner's copy of that half
         int nv = NV;
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) {
             if (nv > 1) {
-                const bool upper = (lane & o) != 0;
                 const int half = nv >> 1;
 #pragma unroll
-                for (int x = 0; x < NV / 2; ++x) {
-                    if (x < half) {
-                        const float send = upper ? v[x] : v[x + half];
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, o);
-                        v[x] = (upper ? v[x + half] : v[x]) + recv;
-                    }
-                }
+                for (int x = 0; x < NV / 2; ++x)
+                    if (x < half) w[x] += __shfl_xor_sync(0xffffffffu, w[x + half], o);
                 nv = half;
             } else {
-                v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+                w[0] += __shfl_xor_sync(0xffffffffu, w[0], o);
             }
         }
-        // lane holds value index = bits of (lane >> (5 - log2 NV)) selected
-        // above: value idx = sum over steps of (upper ? half : 0)
-        int idx = 0, h = NV >> 1;
-#pragma unroll
-        for (int o = 16; o >= 1 && h >= 1; o >>= 1, h >>= 1)
-            if (lane & o) idx += h;
         constexpr int COPIES = 32 / NV;  // lanes holding the same value
         if ((lane & (COPIES - 1)) == 0) {
-            const int r = idx / G, g = idx % G;
-            const int j = j0 + r;
-            if (j <= iabs) srow[(size_t)g * head_stride + j] = v[0] * scale;
+            const int j = j0 + m_r;
+            if (j <= iabs) srow[(size_t)m_g * head_stride + j] = w[0] * scale;
         }
     }
 }
