@@ -256,8 +256,9 @@ __global__ void __launch_bounds__(kBmThreads) blockmean_kernel(KParams p, const 
 // ----------------------------------------------------------------- score ---
 // grid (nqb_max, Hkv, num_seqs), 256 threads.  Pools the valid rows of one
 // query block for the G query heads of one KV head (their rows are
-// contiguous in q), then one warp per key block j <= i_abs forms the G dot
-// products with kbar_j (lanes across d, shuffle reduction).
+// contiguous in q), then each warp takes 4 key blocks j <= i_abs at a time
+// and forms their G dot products with kbar_j (lanes across d, reduce-scatter
+// over the warp).
 template <int D, bool FP8, int G>
 __global__ void __launch_bounds__(256) score_kernel(KParams p, const uint8_t* __restrict__ Q) {
     constexpr int ELT = FP8 ? 1 : 2;
