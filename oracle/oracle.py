@@ -160,6 +160,40 @@ def dense_rows(Q, K, V, rows, heads, mutant: int = 0):
     return out
 
 
+def dense_query_block(Qblk, K, V, p0: int, heads=None):
+    """Causal softmax(QK^T/sqrt(d))V for a block of consecutive query rows, the
+    first at absolute position ``p0`` (row r sees keys ``0 .. p0 + r``), with
+    numpy fp64 matrix products as the steps (the same arithmetic as
+    ``dense_rows``, in the order a matrix product takes): the method with
+    every block kept (tau = +inf) is this dense causal attention, and the
+    product form lets a long sequence be checked block by block.
+    ``Qblk`` [n, Hq, d], ``K``/``V`` [>= p0 + n, Hkv, d]; returns
+    [n * len(heads), d] ordered (row, head), like ``attn_query_block``."""
+    Qblk = _f64(Qblk)
+    n, Hq, d = Qblk.shape
+    Hkv = np.asarray(K).shape[1]
+    G = Hq // Hkv
+    if heads is None:
+        heads = np.arange(Hq, dtype=np.int32)
+    heads = np.asarray(heads, dtype=np.int32)
+    Lk = p0 + n
+    Kd = _f64(np.asarray(K)[:Lk])
+    Vd = _f64(np.asarray(V)[:Lk])
+    # key t is visible to row r iff t <= p0 + r: only the last n keys can be
+    # hidden from a row
+    hidden = np.arange(n)[None, :] > np.arange(n)[:, None]
+    out = np.empty((n, heads.size, d))
+    for c, h in enumerate(heads):
+        hk = h // G
+        z = Qblk[:, h, :] @ Kd[:, hk, :].T
+        z /= np.sqrt(d)
+        z[:, p0:][hidden] = -np.inf
+        z -= z.max(axis=1, keepdims=True)
+        np.exp(z, out=z)
+        out[:, c, :] = (z @ Vd[:, hk, :]) / z.sum(axis=1, keepdims=True)
+    return out.reshape(n * heads.size, d)
+
+
 def all_rows(Lq: int, Hq: int):
     """(rows, heads) covering every query row of every head."""
     t = np.repeat(np.arange(Lq, dtype=np.int32), Hq)

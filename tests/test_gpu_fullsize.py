@@ -129,3 +129,55 @@ def test_full_size(cid, dtype, n_sample):
         assert rows == sum(shape.lens_q) * shape.Hq
     print(f"w{cid}-{dtype}: tau={tau:.4f} drop={drop:.4f} near-threshold pairs={near_total} "
           f"rows compared={rows} (on the GPU's differing mask: {rows_gpu_mask})")
+
+
+# dense runs (every block kept), as the bench times them for its own-dense
+# baseline: too long for the per-row oracle, so query blocks are sampled and
+# the keep-all special case is checked against dense causal attention
+DENSE = [(3, "bf16"), (3, "fp8")]
+DENSE_BLOCKS = 64
+
+
+@pytest.mark.parametrize("cid,dtype", DENSE, ids=[f"w{c}-{d}-dense" for c, d in DENSE])
+def test_full_size_dense(cid, dtype):
+    """tau = +inf at full size: the GPU mask keeps every causal block and the
+    output equals dense causal attention, on 64 seeded query blocks of every
+    sequence's blocks (the last one included), every head of each."""
+    import concurrent.futures as cf
+    import math
+    import os
+    shape = synth.workload(cid, dtype)
+    inp = synth.make_inputs(shape)
+    fp8 = dtype == "fp8"
+    B = shape.B
+    pr = H.problem(inp, out_fill=float("nan"))
+    pr.prefill(math.inf)
+    pr.check()
+    got_bits = H.gpu_bits(pr, inp)
+    rng = np.random.default_rng(777)
+    rows = 0
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        for b in range(inp.num_seqs):
+            Lq, Lk = shape.lens_q[b], shape.lens_k[b]
+            P = Lk - Lq
+            pb, off = P // B, P % B
+            nqb = -(-(off + Lq) // B)
+            # every causal block kept, nothing past the diagonal
+            for i in range(nqb):
+                assert got_bits[b, :, i, : pb + i + 1].all()
+                assert not got_bits[b, :, i, pb + i + 1:].any()
+            K, V = inp.seq_k(b), inp.seq_v(b)
+            picks = sorted({nqb - 1} | set(rng.choice(nqb, size=min(nqb, DENSE_BLOCKS),
+                                                      replace=False).tolist()))
+            a = int(inp.cu_seqlens_q[b])
+            for i in picks:
+                r0, r1 = max(0, i * B - off), min(Lq, (i + 1) * B - off)
+                Qb = inp._deq(inp.q[a + r0: a + r1], inp.q_scale)
+                parts = list(ex.map(lambda h: O.dense_query_block(Qb, K, V, P + r0, [h]),
+                                    range(shape.Hq)))
+                ref = np.stack([x.reshape(r1 - r0, -1) for x in parts], axis=1)
+                got = pr.out[a + r0: a + r1].double().cpu().numpy()
+                H.assert_close(got, ref, fp8, f"w{cid} dense seq {b} block {i}")
+                rows += (r1 - r0) * shape.Hq
+    assert rows >= DENSE_BLOCKS * B * shape.Hq
+    print(f"w{cid}-{dtype} dense: rows compared={rows}")

@@ -77,6 +77,28 @@ def test_dense_routine_matches_torch_sdpa(shape):
 
 
 @pytest.mark.parametrize("shape", SHAPES)
+def test_dense_query_block_matches_the_brute_force(shape):
+    """The matrix-product form of dense causal attention (used to check long
+    dense runs block by block) against the per-row brute force, on every
+    block of each shape, partial first and last blocks included."""
+    Lq, Lk, Hq, Hkv, d, B = shape
+    rng = np.random.default_rng(3)
+    Q, K, V = rand_seq(rng, Lq, Lk, Hq, Hkv, d)
+    P = Lk - Lq
+    rows, heads = O.all_rows(Lq, Hq)
+    ref = O.dense_rows(Q, K, V, rows, heads).reshape(Lq, Hq, d)
+    t = 0
+    while t < Lq:
+        t1 = min(Lq, ((P + t) // B + 1) * B - P)  # the end of the absolute block holding t
+        got = O.dense_query_block(Q[t:t1], K, V, P + t).reshape(t1 - t, Hq, d)
+        np.testing.assert_allclose(got, ref[t:t1], rtol=0, atol=1e-12)
+        sub = np.array([Hq - 1, 0], dtype=np.int32)
+        got_sub = O.dense_query_block(Q[t:t1], K, V, P + t, sub).reshape(t1 - t, 2, d)
+        np.testing.assert_allclose(got_sub, ref[t:t1][:, sub], rtol=0, atol=1e-12)
+        t = t1
+
+
+@pytest.mark.parametrize("shape", SHAPES)
 def test_keep_all_equals_dense(shape):
     Lq, Lk, Hq, Hkv, d, B = shape
     rng = np.random.default_rng(2)
